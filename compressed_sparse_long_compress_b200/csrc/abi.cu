@@ -1,0 +1,260 @@
+// C ABI of libcslc: argument validation, workspace carving and dispatch.
+// Every entry point validates before launching anything and never throws.
+
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace cslc {
+
+static thread_local char g_err[512] = "";
+
+cslc_status set_error(cslc_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+cslc_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return CSLC_OK;
+}
+
+// kernels (defined in the other translation units)
+cslc_status launch_compress(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*,
+                            const uint16_t*, int, int, int, int, uint16_t*, cudaStream_t);
+cslc_status launch_quantize_kv(const uint16_t*, long long, uint8_t*, uint16_t*, float*, cudaStream_t);
+cslc_status launch_indexer_scores(const uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int,
+                                  int, int, int, int, float*, int, cudaStream_t);
+cslc_status launch_topk_rows(const float*, int, int, int, int, int, int, int, int, int, int32_t*,
+                             cudaStream_t);
+cslc_status launch_sparse_attn(const uint16_t*, const uint16_t*, const int32_t*, int, int, int, int, int,
+                               float, uint16_t*, float*, cudaStream_t);
+cslc_status launch_dense_attn(const uint16_t*, const uint16_t*, int, int, int, int, int, int, float,
+                              uint16_t*, float*, cudaStream_t);
+size_t decode_workspace_bytes(const cslc_decode_layer*, int, int, int);
+size_t decode_topk_workspace_bytes(int, int, int);
+cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*, size_t, cudaStream_t);
+cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
+
+constexpr int kMaxTopk = 2048;
+constexpr int kMaxPrefillTopkNc = 49152;   // row of keys must fit in shared memory
+
+static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+#define REQUIRE(cond, st, ...) \
+  do {                          \
+    if (!(cond)) return set_error(st, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(p)                                                                 \
+  do {                                                                                 \
+    REQUIRE((p) != nullptr, CSLC_ERR_NULL, "%s: %s is NULL", __func__, #p);            \
+    REQUIRE(aligned16(p), CSLC_ERR_ALIGN, "%s: %s is not 16-byte aligned", __func__, #p); \
+  } while (0)
+
+// scores rows are processed in blocks of this many rows when the caller does
+// not keep them, so a block stays resident in L2 between the two kernels
+static int score_block_rows(int Nc) {
+  const long long budget = 48ll << 20;   // bytes of scores per block
+  long long rows = budget / ((long long)Nc * 4);
+  rows = rows < 64 ? 64 : rows;
+  rows = (rows / 64) * 64;
+  return (int)rows;
+}
+
+}  // namespace cslc
+
+using namespace cslc;
+
+extern "C" {
+
+int cslc_abi_version(void) { return CSLC_ABI_VERSION; }
+
+const char* cslc_last_error(void) { return g_err; }
+
+cslc_status cslc_sync_status(cslc_stream_t stream) {
+  const cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "cslc_sync_status: %s", cudaGetErrorString(e));
+  return CSLC_OK;
+}
+
+cslc_status csa_compress(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16* c_b,
+                         const cslc_bf16* z_b, const cslc_bf16* pos_bias, int B, int L, int D, int m,
+                         cslc_bf16* out, cslc_stream_t stream) {
+  REQUIRE(B >= 0 && L >= 0, CSLC_ERR_SHAPE, "csa_compress: negative size");
+  REQUIRE(D == kD, CSLC_ERR_UNSUPPORTED, "csa_compress: D must be 128 (got %d)", D);
+  REQUIRE(is_pow2(m) && m <= 128, CSLC_ERR_UNSUPPORTED, "csa_compress: m must be a power of two <= 128");
+  REQUIRE((c_b == nullptr) == (z_b == nullptr), CSLC_ERR_NULL, "csa_compress: give both c_b and z_b or neither");
+  if ((long long)B * (L / m) == 0) return CSLC_OK;
+  REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(pos_bias); REQUIRE_PTR(out);
+  if (c_b) { REQUIRE_PTR(c_b); REQUIRE_PTR(z_b); }
+  return launch_compress(c, z, c_b, z_b, pos_bias, B, L, m, 1, out, stream);
+}
+
+cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16* pos_bias, int B, int L,
+                         int D, int m_prime, cslc_bf16* out, cslc_stream_t stream) {
+  REQUIRE(B >= 0 && L >= 0, CSLC_ERR_SHAPE, "hca_compress: negative size");
+  REQUIRE(D == kD, CSLC_ERR_UNSUPPORTED, "hca_compress: D must be 128 (got %d)", D);
+  REQUIRE(is_pow2(m_prime) && m_prime <= 128, CSLC_ERR_UNSUPPORTED,
+          "hca_compress: m' must be a power of two <= 128");
+  if ((long long)B * (L / m_prime) == 0) return CSLC_OK;
+  REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(pos_bias); REQUIRE_PTR(out);
+  return launch_compress(c, z, nullptr, nullptr, pos_bias, B, L, m_prime, 0, out, stream);
+}
+
+size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {
+  (void)HI; (void)topk;
+  if (scores_given || B <= 0 || L <= 0 || Nc <= 0) return 0;
+  const int rows = score_block_rows(Nc);
+  const int R = L < rows ? L : rows;
+  return (size_t)B * R * Nc * 4;
+}
+
+cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w, const cslc_bf16* k_idx, int B,
+                             int L, int Nc, int HI, int dI, int m, int q_pos0, int topk, float* scores,
+                             int32_t* idx, void* ws, size_t ws_bytes, cslc_stream_t stream) {
+  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE,
+          "csa_indexer_topk: negative size / m < 1");
+  REQUIRE(dI == kDI, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: d_I must be 64 (got %d)", dI);
+  REQUIRE(HI >= 1 && HI <= 16, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: H_I must be in [1, 16]");
+  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: topk must be in [1, 2048]");
+  REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: Nc must be <= %d", kMaxPrefillTopkNc);
+  if ((long long)B * L == 0) return CSLC_OK;
+  REQUIRE_PTR(idx);
+  if (Nc > 0) { REQUIRE_PTR(q_idx); REQUIRE_PTR(w); REQUIRE_PTR(k_idx); }
+  if (scores) REQUIRE_PTR(scores);
+  const size_t need = csa_indexer_topk_workspace_bytes(B, L, Nc, HI, topk, scores != nullptr);
+  if (need) {
+    REQUIRE(ws != nullptr && ws_bytes >= need, CSLC_ERR_WORKSPACE,
+            "csa_indexer_topk: workspace of %zu bytes needed", need);
+    REQUIRE(aligned16(ws), CSLC_ERR_ALIGN, "csa_indexer_topk: ws is not 16-byte aligned");
+  }
+  cslc_status st;
+  if (scores) {
+    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, scores, L, stream);
+    if (st != CSLC_OK) return st;
+    return launch_topk_rows(scores, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
+  }
+  const int R = L < score_block_rows(Nc) ? L : score_block_rows(Nc);
+  float* buf = static_cast<float*>(ws);
+  for (int r0 = 0; r0 < L; r0 += R) {
+    const int r1 = r0 + R < L ? r0 + R : L;
+    if (Nc > 0) {
+      st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, r0, r1, buf, R, stream);
+      if (st != CSLC_OK) return st;
+    }
+    st = launch_topk_rows(buf, R, r0, r1, B, L, Nc, m, q_pos0, topk, idx, stream);
+    if (st != CSLC_OK) return st;
+  }
+  return CSLC_OK;
+}
+
+cslc_status csa_topk(const float* scores, int B, int L, int Nc, int m, int q_pos0, int topk, int32_t* idx,
+                     cslc_stream_t stream) {
+  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE, "csa_topk: bad size");
+  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "csa_topk: topk must be in [1, 2048]");
+  REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "csa_topk: Nc must be <= %d", kMaxPrefillTopkNc);
+  if ((long long)B * L == 0) return CSLC_OK;
+  REQUIRE_PTR(idx);
+  if (Nc > 0) REQUIRE_PTR(scores);
+  return launch_topk_rows(scores, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
+}
+
+cslc_status csa_sparse_attn(const cslc_bf16* q, const cslc_bf16* kv, const int32_t* idx, int B, int L, int H,
+                            int D, int Nc, int topk, float scale, cslc_bf16* out, float* lse,
+                            cslc_stream_t stream) {
+  REQUIRE(B >= 0 && L >= 0 && Nc >= 0, CSLC_ERR_SHAPE, "csa_sparse_attn: negative size");
+  REQUIRE(D == kD, CSLC_ERR_UNSUPPORTED, "csa_sparse_attn: D must be 128");
+  REQUIRE(H >= 16 && H <= 128 && H % 16 == 0, CSLC_ERR_UNSUPPORTED,
+          "csa_sparse_attn: H must be a multiple of 16 in [16, 128]");
+  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "csa_sparse_attn: topk must be in [1, 2048]");
+  if ((long long)B * L == 0) return CSLC_OK;
+  REQUIRE_PTR(q); REQUIRE_PTR(idx); REQUIRE_PTR(out);
+  if (Nc > 0) REQUIRE_PTR(kv);
+  if (lse) REQUIRE_PTR(lse);
+  return launch_sparse_attn(q, kv, idx, B, L, H, Nc, topk, scale, out, lse, stream);
+}
+
+cslc_status hca_dense_attn(const cslc_bf16* q, const cslc_bf16* kv, int B, int L, int H, int D, int Nc,
+                           int m_prime, int q_pos0, float scale, cslc_bf16* out, float* lse,
+                           cslc_stream_t stream) {
+  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m_prime >= 1, CSLC_ERR_SHAPE,
+          "hca_dense_attn: bad size");
+  REQUIRE(D == kD, CSLC_ERR_UNSUPPORTED, "hca_dense_attn: D must be 128");
+  REQUIRE(H >= 16 && H <= 128 && H % 16 == 0, CSLC_ERR_UNSUPPORTED,
+          "hca_dense_attn: H must be a multiple of 16 in [16, 128]");
+  if ((long long)B * L == 0) return CSLC_OK;
+  REQUIRE_PTR(q); REQUIRE_PTR(out);
+  if (Nc > 0) REQUIRE_PTR(kv);
+  if (lse) REQUIRE_PTR(lse);
+  return launch_dense_attn(q, kv, B, L, H, Nc, m_prime, q_pos0, scale, out, lse, stream);
+}
+
+cslc_status cslc_quantize_kv_mixed(const cslc_bf16* kv, int B, int N, uint8_t* nope, cslc_bf16* rope,
+                                   float* scale, cslc_stream_t stream) {
+  REQUIRE(B >= 0 && N >= 0, CSLC_ERR_SHAPE, "cslc_quantize_kv_mixed: negative size");
+  if ((long long)B * N == 0) return CSLC_OK;
+  REQUIRE_PTR(kv); REQUIRE_PTR(nope); REQUIRE_PTR(rope); REQUIRE_PTR(scale);
+  return launch_quantize_kv(kv, (long long)B * N, nope, rope, scale, stream);
+}
+
+size_t cslc_decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers, int B, int H, int HI) {
+  (void)HI;
+  if (layers == nullptr || n_layers <= 0 || B <= 0 || H <= 0) return 0;
+  return decode_workspace_bytes(layers, n_layers, B, H);
+}
+
+cslc_status cslc_decode_step(const cslc_decode_layer* layers, int n_layers, int B, int H, int D, int HI,
+                             int dI, void* ws, size_t ws_bytes, cslc_stream_t stream) {
+  REQUIRE(layers != nullptr || n_layers == 0, CSLC_ERR_NULL, "cslc_decode_step: layers is NULL");
+  REQUIRE(n_layers >= 0 && B >= 0, CSLC_ERR_SHAPE, "cslc_decode_step: negative size");
+  REQUIRE(D == kD && dI == kDI, CSLC_ERR_UNSUPPORTED, "cslc_decode_step: D must be 128 and d_I 64");
+  REQUIRE(H >= 16 && H <= 128 && H % 16 == 0, CSLC_ERR_UNSUPPORTED,
+          "cslc_decode_step: H must be a multiple of 16 in [16, 128]");
+  REQUIRE(HI >= 1 && HI <= 16, CSLC_ERR_UNSUPPORTED, "cslc_decode_step: H_I must be in [1, 16]");
+  if (n_layers == 0 || B == 0) return CSLC_OK;
+  for (int i = 0; i < n_layers; ++i) {
+    const cslc_decode_layer& l = layers[i];
+    REQUIRE(l.kind == 0 || l.kind == 1, CSLC_ERR_UNSUPPORTED, "cslc_decode_step: layer %d kind must be 0 or 1", i);
+    REQUIRE(l.n_max >= 0, CSLC_ERR_SHAPE, "cslc_decode_step: layer %d n_max < 0", i);
+    REQUIRE_PTR(l.q); REQUIRE_PTR(l.out); REQUIRE_PTR(l.n_entries);
+    if (l.n_max > 0) { REQUIRE_PTR(l.nope); REQUIRE_PTR(l.rope); REQUIRE_PTR(l.kv_scale); }
+    if (l.kind == 0) {
+      REQUIRE(l.topk >= 1 && l.topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "cslc_decode_step: layer %d topk", i);
+      if (l.n_max > 0) { REQUIRE_PTR(l.q_idx); REQUIRE_PTR(l.w); REQUIRE_PTR(l.k_idx); }
+      if (l.idx_out) REQUIRE_PTR(l.idx_out);
+      if (l.scores_out) REQUIRE_PTR(l.scores_out);
+    }
+  }
+  const size_t need = decode_workspace_bytes(layers, n_layers, B, H);
+  REQUIRE(ws != nullptr && ws_bytes >= need, CSLC_ERR_WORKSPACE,
+          "cslc_decode_step: workspace of %zu bytes needed", need);
+  REQUIRE(aligned16(ws), CSLC_ERR_ALIGN, "cslc_decode_step: ws is not 16-byte aligned");
+  return run_decode_step(layers, n_layers, B, H, HI, ws, ws_bytes, stream);
+}
+
+size_t cslc_decode_topk_workspace_bytes(int B, int n_max, int topk) {
+  if (B <= 0 || n_max < 0 || topk <= 0) return 0;
+  return decode_topk_workspace_bytes(B, n_max, topk);
+}
+
+cslc_status cslc_decode_topk(const float* scores, const int32_t* n_entries, int B, int n_max, int topk,
+                             int32_t* idx, void* ws, size_t ws_bytes, cslc_stream_t stream) {
+  REQUIRE(B >= 0 && n_max >= 0, CSLC_ERR_SHAPE, "cslc_decode_topk: negative size");
+  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "cslc_decode_topk: topk must be in [1, 2048]");
+  if (B == 0) return CSLC_OK;
+  REQUIRE_PTR(n_entries); REQUIRE_PTR(idx);
+  if (n_max > 0) REQUIRE_PTR(scores);
+  const size_t need = decode_topk_workspace_bytes(B, n_max, topk);
+  REQUIRE(ws != nullptr && ws_bytes >= need, CSLC_ERR_WORKSPACE,
+          "cslc_decode_topk: workspace of %zu bytes needed", need);
+  REQUIRE(aligned16(ws), CSLC_ERR_ALIGN, "cslc_decode_topk: ws is not 16-byte aligned");
+  return run_decode_topk(scores, n_entries, B, n_max, topk, idx, ws, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,690 @@
+// Decode step over the mixed BF16-RoPE / FP8 KV cache.
+//
+// "读完这篇你就搞懂 DeepSeek v4 了", §三: in decode every new token re-reads the
+// compressed KV from HBM, so cost grows with the context; CSA adds the
+// lightning indexer over all entries and attends to the top-k; HCA attends to
+// all entries. First page §1.4 存储格式混: RoPE dims stay BF16, the rest FP8.
+//
+// Kernels (one CSA layer = 1 memset + 5 launches, one HCA layer = 2):
+//   decode_scores_kernel   indexer scores of every entry (tensor-core m16n8k16
+//                          with k_I tiles as A and the 8 indexer heads as N=8),
+//                          ReLU-weighted head sum, fp32 store, and a 4096-bin
+//                          histogram of the score keys (top 12 bits)
+//   decode_select_kernel   finds the histogram bin holding the k-th largest
+//                          score; entries above it are selected, entries in it
+//                          become candidates
+//   decode_finalize_kernel exact choice among the candidates (64-bit radix
+//                          select on score key ++ reversed index, so ties go to
+//                          the smaller index), then a bitonic sort of the k
+//                          indices into ascending order
+//   decode_attn_kernel     split-K attention: each CTA dequantises 256 entries
+//                          (e4m3 * scale -> bf16, RoPE half copied) into shared
+//                          memory and runs QK^T / softmax / PV for all heads
+//   decode_combine_kernel  merges the splits with their max / sum statistics
+
+#include "common.cuh"
+
+namespace cslc {
+
+constexpr int DEC_CHUNK = 4096;      // entries per scores / select CTA
+constexpr int DEC_THREADS = 256;
+constexpr int HIST_BINS = 4096;      // top 12 bits of the score key
+constexpr int HIST_SHIFT = 20;
+constexpr int SPLIT = 256;           // entries per attention CTA
+constexpr int DTILE = 64;            // entries per attention tile
+constexpr int FIN_THREADS = 1024;
+constexpr int MAX_TOPK = 2048;
+
+struct DecodeWs {
+  float* scores;          // [B, n_max]
+  uint32_t* hist;         // [B, HIST_BINS]
+  int32_t* counters;      // [B, 2]: selected-above, candidates
+  int32_t* sel;           // [B, MAX_TOPK]
+  uint2* cand;            // [B, n_max] (key, index)
+  int32_t* idx;           // [B, topk]
+  float* part_o;          // [B, splits, H, 128]
+  float* part_ml;         // [B, splits, H, 2]
+};
+
+// ------------------------------------------------------------ scores + hist
+
+template <int NT>  // indexer heads padded to NT * 8
+__global__ void __launch_bounds__(DEC_THREADS) decode_scores_kernel(
+    const uint16_t* __restrict__ q_idx, const uint16_t* __restrict__ w,
+    const uint16_t* __restrict__ k_idx, const int32_t* __restrict__ n_entries, int n_max, int HI,
+    float* __restrict__ scores, uint32_t* __restrict__ ghist) {
+  __shared__ uint32_t hist[HIST_BINS];
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const int n = min(n_entries[b], n_max);
+  const int c0 = blockIdx.x * DEC_CHUNK;
+  if (c0 >= n) return;   // whole CTA exits together: no barrier reached
+  for (int x = tid; x < HIST_BINS; x += DEC_THREADS) hist[x] = 0;
+
+  // B fragments: q_I of head nt*8+g, physical dims 16*tq .. 16*tq+15 (see the
+  // dims permutation note below); weights of heads nt*8 + 2*tq, +1.
+  uint32_t qb[NT][8];
+  float wv[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int h = nt * 8 + g;
+    if (h < HI) {
+      const uint4* src = reinterpret_cast<const uint4*>(q_idx + ((size_t)b * HI + h) * kDI + 16 * tq);
+      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      qb[nt][0] = v0.x; qb[nt][1] = v0.y; qb[nt][2] = v0.z; qb[nt][3] = v0.w;
+      qb[nt][4] = v1.x; qb[nt][5] = v1.y; qb[nt][6] = v1.z; qb[nt][7] = v1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) qb[nt][j] = 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hw = nt * 8 + 2 * tq + j;
+      wv[nt][j] = hw < HI ? bf16_to_f(w[(size_t)b * HI + hw]) : 0.f;
+    }
+  }
+  __syncthreads();
+
+  // Dims permutation: the product runs over the 64 dims in any order as long
+  // as A and B agree. Thread (g, tq) loads physical dims [16tq, 16tq+16) of
+  // rows g and g+8; in k-step s its fragment registers hold physical pairs
+  // 16tq+4s (+0,+1) and 16tq+4s+2 (+2,+3) -- the same pairs its B registers hold.
+  const int c1 = min(n, c0 + DEC_CHUNK);
+  const uint16_t* kbase = k_idx + (size_t)b * n_max * kDI;
+  for (int e0 = c0 + warp * 16; e0 < c1; e0 += 16 * (DEC_THREADS / 32)) {
+    const int ea = e0 + g, eb = ea + 8;
+    uint32_t ra[8], rb[8];
+    {
+      const uint4* pa = reinterpret_cast<const uint4*>(kbase + (size_t)min(ea, n - 1) * kDI + 16 * tq);
+      const uint4* pb = reinterpret_cast<const uint4*>(kbase + (size_t)min(eb, n - 1) * kDI + 16 * tq);
+      const uint4 a0 = __ldcs(pa), a1 = __ldcs(pa + 1), b0 = __ldcs(pb), b1 = __ldcs(pb + 1);
+      ra[0] = a0.x; ra[1] = a0.y; ra[2] = a0.z; ra[3] = a0.w; ra[4] = a1.x; ra[5] = a1.y; ra[6] = a1.z; ra[7] = a1.w;
+      rb[0] = b0.x; rb[1] = b0.y; rb[2] = b0.z; rb[3] = b0.w; rb[4] = b1.x; rb[5] = b1.y; rb[6] = b1.z; rb[7] = b1.w;
+    }
+    float sa = 0.f, sb = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t af[4] = {ra[2 * s], rb[2 * s], ra[2 * s + 1], rb[2 * s + 1]};
+        mma_bf16_16816(d, af, qb[nt][2 * s], qb[nt][2 * s + 1]);
+      }
+      sa = fmaf(wv[nt][0], fmaxf(d[0], 0.f), sa);
+      sa = fmaf(wv[nt][1], fmaxf(d[1], 0.f), sa);
+      sb = fmaf(wv[nt][0], fmaxf(d[2], 0.f), sb);
+      sb = fmaf(wv[nt][1], fmaxf(d[3], 0.f), sb);
+    }
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+    // lane tq==0 owns row g, lane tq==1 owns row g+8
+    const int e = tq == 0 ? ea : eb;
+    const float v = tq == 0 ? sa : sb;
+    const bool mine = tq < 2 && e < c1;
+    if (mine) scores[(size_t)b * n_max + e] = v;
+    if (mine) {
+      const uint32_t bin = float_key(v) >> HIST_SHIFT;
+      const unsigned peers = __match_any_sync(__activemask(), bin);
+      if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+  }
+  __syncthreads();
+  uint32_t* gh = ghist + (size_t)b * HIST_BINS;
+  for (int x = tid; x < HIST_BINS; x += DEC_THREADS) {
+    const uint32_t v = hist[x];
+    if (v) atomicAdd(&gh[x], v);
+  }
+}
+
+// Histogram only (for the stand-alone top-k entry on given scores).
+__global__ void __launch_bounds__(DEC_THREADS) decode_hist_kernel(const float* __restrict__ scores,
+                                                                  const int32_t* __restrict__ n_entries,
+                                                                  int n_max, uint32_t* __restrict__ ghist) {
+  __shared__ uint32_t hist[HIST_BINS];
+  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int n = min(n_entries[b], n_max);
+  const int c0 = blockIdx.x * DEC_CHUNK;
+  if (c0 >= n) return;
+  for (int x = tid; x < HIST_BINS; x += DEC_THREADS) hist[x] = 0;
+  __syncthreads();
+  const int c1 = min(n, c0 + DEC_CHUNK);
+  for (int e = c0 + tid; e < c1; e += DEC_THREADS) {
+    const uint32_t bin = float_key(scores[(size_t)b * n_max + e]) >> HIST_SHIFT;
+    const unsigned peers = __match_any_sync(__activemask(), bin);
+    if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+  }
+  __syncthreads();
+  for (int x = tid; x < HIST_BINS; x += DEC_THREADS) {
+    const uint32_t v = hist[x];
+    if (v) atomicAdd(&ghist[(size_t)b * HIST_BINS + x], v);
+  }
+}
+
+// -------------------------------------------------------------- selection
+
+// Finds bin T with count(bins > T) < k <= count(bins >= T). Block-wide, DEC_THREADS.
+__device__ void find_threshold_bin(const uint32_t* gh, int k, int* out_bin, int* out_above) {
+  __shared__ uint32_t part[DEC_THREADS];
+  const int tid = threadIdx.x;
+  // thread t owns bins 4095-16t .. 4080-16t
+  uint32_t cnt[16], s = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) { cnt[j] = gh[HIST_BINS - 1 - 16 * tid - j]; s += cnt[j]; }
+  part[tid] = s;
+  __syncthreads();
+  // inclusive scan over threads (Hillis-Steele in shared memory)
+  for (int o = 1; o < DEC_THREADS; o <<= 1) {
+    const uint32_t v = tid >= o ? part[tid - o] : 0u;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  const uint32_t incl = part[tid], excl = incl - s;
+  if (excl < (uint32_t)k && incl >= (uint32_t)k) {
+    uint32_t above = excl;
+    for (int j = 0; j < 16; ++j) {
+      if (above + cnt[j] >= (uint32_t)k) {
+        *out_bin = HIST_BINS - 1 - 16 * tid - j;
+        *out_above = (int)above;
+        break;
+      }
+      above += cnt[j];
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
+    const float* __restrict__ scores, const int32_t* __restrict__ n_entries, int n_max, int topk,
+    const uint32_t* __restrict__ ghist, int32_t* __restrict__ counters, int32_t* __restrict__ sel,
+    uint2* __restrict__ cand) {
+  __shared__ int thr[2];
+  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  if (tid == 0) { thr[0] = HIST_BINS; thr[1] = 0; }   // "nothing above" if no bin is found
+  const int n = min(n_entries[b], n_max);
+  const int c0 = blockIdx.x * DEC_CHUNK;
+  if (n <= topk || c0 >= n) return;
+  find_threshold_bin(ghist + (size_t)b * HIST_BINS, topk, &thr[0], &thr[1]);
+  const uint32_t T = (uint32_t)thr[0];
+  const int c1 = min(n, c0 + DEC_CHUNK);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = c0; base < c1; base += DEC_THREADS) {
+    const int e = base + tid;
+    const bool valid = e < c1;
+    const uint32_t key = valid ? float_key(scores[(size_t)b * n_max + e]) : 0u;
+    const uint32_t bin = key >> HIST_SHIFT;
+    const bool above = valid && bin > T, inbin = valid && bin == T;
+    const unsigned ma = __ballot_sync(0xffffffffu, above);
+    const unsigned mc = __ballot_sync(0xffffffffu, inbin);
+    int base_a = 0, base_c = 0;
+    if (lane == 0) {
+      if (ma) base_a = atomicAdd(&counters[2 * b], __popc(ma));
+      if (mc) base_c = atomicAdd(&counters[2 * b + 1], __popc(mc));
+    }
+    base_a = __shfl_sync(0xffffffffu, base_a, 0);
+    base_c = __shfl_sync(0xffffffffu, base_c, 0);
+    const int pa = base_a + __popc(ma & lt), pc = base_c + __popc(mc & lt);
+    if (above && pa < MAX_TOPK) sel[(size_t)b * MAX_TOPK + pa] = e;
+    if (inbin && pc < n_max) cand[(size_t)b * n_max + pc] = make_uint2(key, (uint32_t)e);
+  }
+}
+
+// 64-bit composite of a candidate: score key, then reversed index, so that a
+// larger composite means a larger score or an equal score at a smaller index.
+__device__ __forceinline__ uint64_t cand_key(uint2 c) {
+  return ((uint64_t)c.x << 32) | (uint64_t)(0xffffffffu - c.y);
+}
+
+__global__ void __launch_bounds__(FIN_THREADS) decode_finalize_kernel(
+    const int32_t* __restrict__ n_entries, int n_max, int topk, const int32_t* __restrict__ counters,
+    const int32_t* __restrict__ sel, const uint2* __restrict__ cand, int32_t* __restrict__ idx) {
+  __shared__ int32_t list[MAX_TOPK];
+  __shared__ uint32_t hist[FIN_THREADS / 32][256];
+  __shared__ int bc[4];
+  __shared__ int fill;
+  const int b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = min(n_entries[b], n_max);
+  int32_t* out = idx + (size_t)b * topk;
+  if (n <= topk) {
+    for (int j = tid; j < topk; j += FIN_THREADS) out[j] = j < n ? j : -1;
+    return;
+  }
+  const int n_above = min(counters[2 * b], topk);
+  const int C = min(counters[2 * b + 1], n_max);
+  const int need = topk - n_above;
+  const uint2* cb = cand + (size_t)b * n_max;
+  for (int j = tid; j < n_above; j += FIN_THREADS) list[j] = sel[(size_t)b * MAX_TOPK + j];
+  if (tid == 0) fill = n_above;
+  __syncthreads();
+
+  // radix select of the need-th largest composite key among the C candidates
+  uint64_t prefix = 0, mask = 0;
+  int remaining = need;
+  bool take_all = (C == need);
+  for (int shift = 56; shift >= 0 && !take_all; shift -= 8) {
+    for (int x = tid; x < (FIN_THREADS / 32) * 256; x += FIN_THREADS) (&hist[0][0])[x] = 0;
+    if (tid == 0) { bc[0] = 0; bc[1] = 0; bc[2] = 0; }
+    __syncthreads();
+    for (int i = tid; i < C; i += FIN_THREADS) {
+      const uint64_t k = cand_key(cb[i]);
+      if ((k & mask) == prefix) {
+        const uint32_t d = (uint32_t)(k >> shift) & 255u;
+        const unsigned peers = __match_any_sync(__activemask(), d);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp][d], (uint32_t)__popc(peers));
+      }
+    }
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t s = 0;
+      for (int w = 0; w < FIN_THREADS / 32; ++w) s += hist[w][tid];
+      hist[0][tid] = s;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t cnt[8], ls = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cnt[j] = hist[0][255 - 8 * lane - j]; ls += cnt[j]; }
+      uint32_t incl = ls;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t excl = incl - ls;
+      if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
+        uint32_t above = excl;
+        for (int j = 0; j < 8; ++j) {
+          if (above + cnt[j] >= (uint32_t)remaining) {
+            bc[0] = 255 - 8 * lane - j; bc[1] = (int)above; bc[2] = (int)cnt[j];
+            break;
+          }
+          above += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    const uint64_t d = (uint64_t)bc[0];
+    const int above = bc[1], cnt_d = bc[2];
+    __syncthreads();
+    remaining -= above;
+    prefix |= d << shift;
+    mask |= 255ull << shift;
+    if (cnt_d == remaining) take_all = true;
+  }
+  // composite keys are unique, so after the last digit exactly `remaining` match
+  for (int i = tid; i < C; i += FIN_THREADS) {
+    const uint2 c = cb[i];
+    const uint64_t k = cand_key(c);
+    const bool s = take_all ? ((k & mask) >= prefix) : ((k & mask) > prefix || (k & mask) == prefix);
+    if (s) {
+      const int pos = atomicAdd(&fill, 1);
+      if (pos < topk) list[pos] = (int32_t)c.y;
+    }
+  }
+  __syncthreads();
+  // bitonic sort of list[0..topk) ascending, padded to a power of two
+  int P = 1;
+  while (P < topk) P <<= 1;
+  for (int j = topk + tid; j < P; j += FIN_THREADS) list[j] = 0x7fffffff;
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < P; i += FIN_THREADS) {
+        const int jx = i ^ stride;
+        if (jx > i) {
+          const bool up = (i & size) == 0;
+          const int a = list[i], c = list[jx];
+          if ((a > c) == up) { list[i] = c; list[jx] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int j = tid; j < topk; j += FIN_THREADS) out[j] = list[j];
+}
+
+// -------------------------------------------------------------- attention
+
+template <bool SPARSE>
+__global__ void __launch_bounds__(256) decode_attn_kernel(
+    const uint16_t* __restrict__ q, const uint8_t* __restrict__ nope, const uint16_t* __restrict__ rope,
+    const float* __restrict__ kv_scale, const int32_t* __restrict__ n_entries, int n_max,
+    const int32_t* __restrict__ idx, int topk, int H, float scale_log2, int splits,
+    float* __restrict__ part_o, float* __restrict__ part_ml) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* q_s = smem;                       // [H][256 B]
+  uint8_t* kv_s = smem + H * 256;            // [DTILE][256 B]
+  __shared__ int32_t ent[SPLIT];
+  const int b = blockIdx.y, sp = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nthreads = (H / 16) * 32;
+  const int g = lane >> 2, tq = lane & 3;
+  const int n = min(n_entries[b], n_max);
+  const int s0 = sp * SPLIT;
+  const int n_slots = SPARSE ? topk : n;
+
+  for (int x = tid; x < H * 16; x += nthreads) {
+    const int chunk = x & 15, row = x >> 4;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)b * H + row) * kD) + chunk);
+    *reinterpret_cast<uint4*>(q_s + swz(row, chunk, 256)) = v;
+  }
+  for (int j = tid; j < SPLIT; j += nthreads) {
+    const int slot = s0 + j;
+    int e = -1;
+    if (slot < n_slots) e = SPARSE ? idx[(size_t)b * topk + slot] : slot;
+    if (e >= n) e = -1;
+    ent[j] = e;
+  }
+  __syncthreads();
+  uint32_t qf[8][4];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int row = warp * 16 + (lane & 15);
+    const int chunk = ks * 2 + (lane >> 4);
+    ldsm_x4(smem_u32(q_s + swz(row, chunk, 256)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+  }
+  float o[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+
+  for (int t0 = 0; t0 < SPLIT; t0 += DTILE) {
+    if (s0 + t0 >= n_slots) break;
+    // dequantise 64 entries into shared memory: chunks 0..7 FP8 dims, 8..15 RoPE dims
+    for (int x = tid; x < DTILE * 16; x += nthreads) {
+      const int chunk = x & 15, row = x >> 4;
+      const int e = ent[t0 + row];
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (e >= 0) {
+        const size_t er = (size_t)b * n_max + e;
+        if (chunk < 8) {
+          const uint2 c8 = __ldg(reinterpret_cast<const uint2*>(nope + er * kNope) + chunk);
+          const float sc = __ldg(kv_scale + er);
+          const uint32_t cw[2] = {c8.x, c8.y};
+          uint32_t ow[4];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] & 0xffffu), __NV_E4M3);
+            const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] >> 16), __NV_E4M3);
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+            ow[2 * k] = pack_bf16x2(f01.x * sc, f01.y * sc);
+            ow[2 * k + 1] = pack_bf16x2(f23.x * sc, f23.y * sc);
+          }
+          v = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        } else {
+          v = __ldg(reinterpret_cast<const uint4*>(rope + er * kRope) + (chunk - 8));
+        }
+      }
+      *reinterpret_cast<uint4*>(kv_s + swz(row, chunk, 256)) = v;
+    }
+    __syncthreads();
+    float s[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[i][j] = 0.f;
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t b0, b1, b2, b3;
+        const int row = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int chunk = ks * 2 + ((lane >> 3) & 1);
+        ldsm_x4(smem_u32(kv_s + swz(row, chunk, 256)), b0, b1, b2, b3);
+        mma_bf16_16816(s[2 * np], qf[ks], b0, b1);
+        mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
+      }
+    }
+    float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const bool valid = ent[t0 + nt * 8 + 2 * tq + j] >= 0;
+        const float v0 = valid ? s[nt][j] * scale_log2 : -INFINITY;
+        const float v1 = valid ? s[nt][2 + j] * scale_log2 : -INFINITY;
+        s[nt][j] = v0;
+        s[nt][2 + j] = v1;
+        tmax[0] = fmaxf(tmax[0], v0);
+        tmax[1] = fmaxf(tmax[1], v1);
+      }
+    }
+    float alpha[2], mnew[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
+      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
+      mnew[r] = fmaxf(mrow[r], tmax[r]);
+      alpha[r] = mrow[r] == -INFINITY ? 0.f : exp2f(mrow[r] - mnew[r]);
+      mrow[r] = mnew[r];
+    }
+    float psum[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = j >> 1;
+        const float p = mnew[r] == -INFINITY ? 0.f : exp2f(s[nt][j] - mnew[r]);
+        s[nt][j] = p;
+        psum[r] += p;
+      }
+    }
+    lrow[0] = lrow[0] * alpha[0] + psum[0];
+    lrow[1] = lrow[1] * alpha[1] + psum[1];
+#pragma unroll
+    for (int dn = 0; dn < 16; ++dn) {
+      o[dn][0] *= alpha[0]; o[dn][1] *= alpha[0];
+      o[dn][2] *= alpha[1]; o[dn][3] *= alpha[1];
+    }
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
+      pa[1] = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
+      pa[2] = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+      pa[3] = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+      for (int dp = 0; dp < 8; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        const int row = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int chunk = dp * 2 + (lane >> 4);
+        ldsm_x4_t(smem_u32(kv_s + swz(row, chunk, 256)), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * dp], pa, b0, b1);
+        mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
+    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
+  }
+  const int h0 = warp * 16 + g, h1 = h0 + 8;
+  float* po = part_o + (((size_t)b * splits + sp) * H) * kD;
+#pragma unroll
+  for (int dn = 0; dn < 16; ++dn) {
+    const int col = dn * 8 + 2 * tq;
+    *reinterpret_cast<float2*>(po + (size_t)h0 * kD + col) = make_float2(o[dn][0], o[dn][1]);
+    *reinterpret_cast<float2*>(po + (size_t)h1 * kD + col) = make_float2(o[dn][2], o[dn][3]);
+  }
+  if (tq == 0) {
+    float* pm = part_ml + (((size_t)b * splits + sp) * H) * 2;
+    pm[2 * h0] = mrow[0]; pm[2 * h0 + 1] = lrow[0];
+    pm[2 * h1] = mrow[1]; pm[2 * h1 + 1] = lrow[1];
+  }
+}
+
+__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_ml,
+                                                             const int32_t* __restrict__ n_entries,
+                                                             int n_max, int topk, int sparse, int H,
+                                                             int splits, uint16_t* __restrict__ out) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int n = min(n_entries[b], n_max);
+  const int used = sparse ? min(splits, (min(topk, n) + SPLIT - 1) / SPLIT) : min(splits, (n + SPLIT - 1) / SPLIT);
+  const float* pm = part_ml + (size_t)b * splits * H * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < used; ++s) M = fmaxf(M, pm[((size_t)s * H + h) * 2]);
+  float num = 0.f, den = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < used; ++s) {
+      const float ms = pm[((size_t)s * H + h) * 2];
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      den = fmaf(f, pm[((size_t)s * H + h) * 2 + 1], den);
+      num = fmaf(f, part_o[(((size_t)b * splits + s) * H + h) * kD + d], num);
+    }
+  }
+  const float r = den > 0.f ? num / den : 0.f;
+  out[((size_t)b * H + h) * kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+}
+
+// -------------------------------------------------------------- host side
+
+static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct DecodeWsSizes {
+  size_t scores, hist, counters, sel, cand, idx, part_o, part_ml;
+  size_t total() const { return scores + hist + counters + sel + cand + idx + part_o + part_ml; }
+};
+
+static int layer_splits(const cslc_decode_layer& l) {
+  const int slots = l.kind == 0 ? l.topk : l.n_max;
+  return slots > 0 ? (slots + SPLIT - 1) / SPLIT : 1;
+}
+
+static DecodeWsSizes ws_sizes(int B, int n_max, int topk, int splits, int H) {
+  DecodeWsSizes s;
+  s.scores = align_up((size_t)B * n_max * 4);
+  s.hist = align_up((size_t)B * HIST_BINS * 4);
+  s.counters = align_up((size_t)B * 2 * 4);
+  s.sel = align_up((size_t)B * MAX_TOPK * 4);
+  s.cand = align_up((size_t)B * n_max * 8);
+  s.idx = align_up((size_t)B * (topk > 0 ? topk : 1) * 4);
+  s.part_o = align_up((size_t)B * splits * H * kD * 4);
+  s.part_ml = align_up((size_t)B * splits * H * 2 * 4);
+  return s;
+}
+
+size_t decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers, int B, int H) {
+  size_t best = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    const cslc_decode_layer& l = layers[i];
+    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l), H);
+    if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
+    best = s.total() > best ? s.total() : best;
+  }
+  return best;
+}
+
+size_t decode_topk_workspace_bytes(int B, int n_max, int topk) {
+  DecodeWsSizes s = ws_sizes(B, n_max, topk, 1, 16);
+  return s.hist + s.counters + s.sel + s.cand;
+}
+
+static void carve(uint8_t* base, const DecodeWsSizes& s, DecodeWs& w) {
+  uint8_t* p = base;
+  w.hist = reinterpret_cast<uint32_t*>(p); p += s.hist;
+  w.counters = reinterpret_cast<int32_t*>(p); p += s.counters;
+  w.scores = reinterpret_cast<float*>(p); p += s.scores;
+  w.sel = reinterpret_cast<int32_t*>(p); p += s.sel;
+  w.cand = reinterpret_cast<uint2*>(p); p += s.cand;
+  w.idx = reinterpret_cast<int32_t*>(p); p += s.idx;
+  w.part_o = reinterpret_cast<float*>(p); p += s.part_o;
+  w.part_ml = reinterpret_cast<float*>(p); p += s.part_ml;
+}
+
+static cslc_status run_topk_stages(const float* scores, const int32_t* n_entries, int B, int n_max,
+                                   int topk, DecodeWs& w, int32_t* idx, cudaStream_t stream) {
+  const dim3 grid((n_max + DEC_CHUNK - 1) / DEC_CHUNK, B);
+  if (n_max > 0) {
+    decode_select_kernel<<<grid, DEC_THREADS, 0, stream>>>(scores, n_entries, n_max, topk, w.hist,
+                                                           w.counters, w.sel, w.cand);
+    cslc_status st = check_launch("decode_select_kernel");
+    if (st != CSLC_OK) return st;
+  }
+  decode_finalize_kernel<<<B, FIN_THREADS, 0, stream>>>(n_entries, n_max, topk, w.counters, w.sel,
+                                                        w.cand, idx);
+  return check_launch("decode_finalize_kernel");
+}
+
+static cslc_status run_attention(const cslc_decode_layer& l, int B, int H, const int32_t* idx,
+                                 DecodeWs& w, cudaStream_t stream) {
+  const int splits = layer_splits(l);
+  const size_t smem = (size_t)H * 256 + DTILE * 256;
+  const dim3 grid(splits, B);
+  const float sl2 = l.scale * kLog2e;
+  if (l.kind == 0)
+    decode_attn_kernel<true><<<grid, (H / 16) * 32, smem, stream>>>(
+        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, idx, l.topk, H, sl2, splits, w.part_o, w.part_ml);
+  else
+    decode_attn_kernel<false><<<grid, (H / 16) * 32, smem, stream>>>(
+        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, nullptr, 0, H, sl2, splits, w.part_o, w.part_ml);
+  cslc_status st = check_launch("decode_attn_kernel");
+  if (st != CSLC_OK) return st;
+  decode_combine_kernel<<<dim3(H, B), kD, 0, stream>>>(w.part_o, w.part_ml, l.n_entries, l.n_max, l.topk,
+                                                       l.kind == 0, H, splits, l.out);
+  return check_launch("decode_combine_kernel");
+}
+
+cslc_status run_decode_step(const cslc_decode_layer* layers, int n_layers, int B, int H, int HI,
+                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+  for (int i = 0; i < n_layers; ++i) {
+    const cslc_decode_layer& l = layers[i];
+    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l), H);
+    if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
+    DecodeWs w;
+    carve(static_cast<uint8_t*>(ws), s, w);
+    cslc_status st;
+    if (l.kind == 0) {
+      float* scores = l.scores_out ? l.scores_out : w.scores;
+      int32_t* idx = l.idx_out ? l.idx_out : w.idx;
+      if (cudaMemsetAsync(w.hist, 0, s.hist + s.counters, stream) != cudaSuccess)
+        return set_error(CSLC_ERR_CUDA, "cudaMemsetAsync failed");
+      if (l.n_max > 0) {
+        const dim3 grid((l.n_max + DEC_CHUNK - 1) / DEC_CHUNK, B);
+        if (HI <= 8)
+          decode_scores_kernel<1><<<grid, DEC_THREADS, 0, stream>>>(l.q_idx, l.w, l.k_idx, l.n_entries,
+                                                                    l.n_max, HI, scores, w.hist);
+        else
+          decode_scores_kernel<2><<<grid, DEC_THREADS, 0, stream>>>(l.q_idx, l.w, l.k_idx, l.n_entries,
+                                                                    l.n_max, HI, scores, w.hist);
+        st = check_launch("decode_scores_kernel");
+        if (st != CSLC_OK) return st;
+      }
+      st = run_topk_stages(scores, l.n_entries, B, l.n_max, l.topk, w, idx, stream);
+      if (st != CSLC_OK) return st;
+      st = run_attention(l, B, H, idx, w, stream);
+    } else {
+      st = run_attention(l, B, H, nullptr, w, stream);
+    }
+    if (st != CSLC_OK) return st;
+  }
+  return CSLC_OK;
+}
+
+cslc_status run_decode_topk(const float* scores, const int32_t* n_entries, int B, int n_max, int topk,
+                            int32_t* idx, void* ws, cudaStream_t stream) {
+  DecodeWsSizes s = ws_sizes(B, n_max, topk, 1, 16);
+  s.scores = s.idx = s.part_o = s.part_ml = 0;
+  DecodeWs w;
+  carve(static_cast<uint8_t*>(ws), s, w);
+  if (cudaMemsetAsync(w.hist, 0, s.hist + s.counters, stream) != cudaSuccess)
+    return set_error(CSLC_ERR_CUDA, "cudaMemsetAsync failed");
+  if (n_max > 0) {
+    const dim3 grid((n_max + DEC_CHUNK - 1) / DEC_CHUNK, B);
+    decode_hist_kernel<<<grid, DEC_THREADS, 0, stream>>>(scores, n_entries, n_max, w.hist);
+    cslc_status st = check_launch("decode_hist_kernel");
+    if (st != CSLC_OK) return st;
+  }
+  return run_topk_stages(scores, n_entries, B, n_max, topk, w, idx, stream);
+}
+
+}  // namespace cslc

@@ -1,0 +1,226 @@
+/*
+ * cslc.h -- C ABI of the hybrid compressed attention library (libcslc.so).
+ *
+ * The library implements the attention path of the CSA / HCA hybrid layer
+ * described on the DeepSeek-V4 explainer pages:
+ *   CSA  ("从论文出发，逐层剖析 CSA / HCA 混注意力…", §1.1 and its 工程细节 paragraph;
+ *         "读完这篇你就搞懂 DeepSeek v4 了", §三 CSA steps 1-3): every m=4 tokens become
+ *         one KV entry compressed from an overlapped 2m-token window, a lightning
+ *         indexer scores every entry per query, the top-k (1024) entries are
+ *         selected, and all query heads attend to that selection with one KV head.
+ *   HCA  (same pages, §1.2 / HCA 步骤简化): every m'=128 tokens become one entry,
+ *         followed by dense causal attention over the short sequence.
+ *   Decode KV layout (first page, §1.4 存储格式混): RoPE dims in BF16, the other
+ *         dims in FP8 (e4m3) with one fp32 scale per entry.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates or frees device memory. Scratch memory comes from a
+ *     caller-provided workspace whose size the matching *_workspace_bytes()
+ *     function reports (returns 0 when none is needed).
+ *   - Tensors are dense, row-major (last index fastest) with the shapes given
+ *     below. bf16 tensors are passed as cslc_bf16 (raw bfloat16 bits).
+ *     Every pointer must be 16-byte aligned (CSLC_ERR_ALIGN otherwise).
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and
+ *     return after the launches are enqueued. Arguments are validated before
+ *     anything is launched: on any error status nothing has been written.
+ *     Errors from the CUDA launch itself return CSLC_ERR_CUDA.
+ *   - No exception or abort crosses the ABI. cslc_last_error() returns a
+ *     thread-local text for the last non-OK status.
+ *   - Supported shapes: D = 128 (compressed entry / head dim), d_I = 64, H a
+ *     multiple of 16 up to 128, H_I <= 16, 1 <= topk <= 2048, m a power of two
+ *     in [1, 128] for compression (any m >= 1 for visibility). Anything else
+ *     returns CSLC_ERR_UNSUPPORTED.
+ *
+ * Geometry shared by every call (the pages leave it open; this is the reading
+ * the library follows): entry i of a compression with ratio m covers the
+ * tokens up to position (i+1)m-1; a query at absolute position p sees entry i
+ * iff (i+1)m-1 <= p, so n_vis(p) = min(N_c, floor((p+1)/m)). Only complete
+ * windows are compressed: N_c = floor(L/m).
+ */
+#ifndef CSLC_H_
+#define CSLC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSLC_ABI_VERSION 1
+
+typedef uint16_t cslc_bf16;              /* raw bfloat16 bits */
+typedef struct CUstream_st* cslc_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  CSLC_OK = 0,
+  CSLC_ERR_NULL = 1,          /* a required pointer is NULL */
+  CSLC_ERR_SHAPE = 2,         /* a size is negative / inconsistent */
+  CSLC_ERR_ALIGN = 3,         /* a pointer is not 16-byte aligned */
+  CSLC_ERR_UNSUPPORTED = 4,   /* shape outside the supported set */
+  CSLC_ERR_WORKSPACE = 5,     /* workspace missing or too small */
+  CSLC_ERR_CUDA = 6,          /* a CUDA call or launch failed */
+  CSLC_ERR_DEVICE_CHECK = 7   /* a kernel's own check failed (see cslc_sync_status) */
+} cslc_status;
+
+/* Version of this ABI (CSLC_ABI_VERSION). Never fails. */
+int cslc_abi_version(void);
+
+/* Text of the last non-OK status returned on the calling thread. */
+const char* cslc_last_error(void);
+
+/* Waits for `stream`, then reports (and clears) any error a kernel recorded in
+ * its device-side status word; returns CSLC_OK when none. */
+cslc_status cslc_sync_status(cslc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Compression ("读完这篇你就搞懂 DeepSeek v4 了", §三 压缩机制; first page §1.1 工程细节)
+ *
+ * For entry i and channel j:
+ *   e_i[j] = sum_{t in W_i} softmax_t( z_t[j] + pos_bias[slot(t)][j] ) * c_t[j]
+ * computed in fp32, stored bf16 (round to nearest even).
+ * CSA window W_i: C^b = tokens (i-1)m .. im-1 in slots 0..m-1 (absent for
+ * i = 0) and C^a = tokens im .. im+m-1 in slots m..2m-1.
+ *
+ *   c, z      [B, L, D] bf16  candidate vectors and compression logits
+ *   c_b, z_b  [B, L, D] bf16  optional separate streams read for the C^b half;
+ *                             pass both NULL to read c, z there too
+ *   pos_bias  [2m, D] bf16    positional bias per window slot
+ *   out       [B, floor(L/m), D] bf16
+ * Requires D == 128, m a power of two in [1, 128]. L < m gives 0 entries
+ * (nothing launched).
+ */
+cslc_status csa_compress(const cslc_bf16* c, const cslc_bf16* z,
+                         const cslc_bf16* c_b, const cslc_bf16* z_b,
+                         const cslc_bf16* pos_bias, int B, int L, int D, int m,
+                         cslc_bf16* out, cslc_stream_t stream);
+
+/* HCA compression (first page §1.2; "读完这篇…" §三 HCA 步骤简化): one window of
+ * m' tokens per entry, no overlap: W_i = tokens im' .. im'+m'-1, slot = t - im'.
+ *   pos_bias [m', D] bf16; out [B, floor(L/m'), D] bf16. */
+cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z,
+                         const cslc_bf16* pos_bias, int B, int L, int D,
+                         int m_prime, cslc_bf16* out, cslc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Lightning indexer + top-k ("读完这篇…" §三 闪电索引; first page §1.1 top-k=1024)
+ *
+ *   S[b,t,i] = sum_h w[b,t,h] * max(0, q_idx[b,t,h,:] . k_idx[b,i,:])
+ * for the entries visible to query row t (absolute position q_pos0 + t),
+ * computed with fp32 accumulation of bf16 products and stored fp32.
+ * idx[b,t,:] = the min(topk, n_vis) visible entries with the largest S (ties
+ * to the smaller entry index), in ascending index order, then -1 padding.
+ *
+ *   q_idx  [B, L, H_I, d_I] bf16     w [B, L, H_I] bf16     k_idx [B, Nc, d_I] bf16
+ *   scores [B, L, Nc] fp32 or NULL.  When given, row t holds S for entries
+ *          0..n_vis(t)-1; entries from n_vis(t) on are left unspecified.
+ *          When NULL the scores live only in the workspace, in row blocks.
+ *   idx    [B, L, topk] int32
+ *   ws     workspace of csa_indexer_topk_workspace_bytes() bytes (may be NULL
+ *          when that is 0).
+ * Requires d_I == 64, 1 <= H_I <= 16, 1 <= topk <= 2048, q_pos0 >= 0.
+ */
+size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given);
+cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w,
+                             const cslc_bf16* k_idx, int B, int L, int Nc, int HI,
+                             int dI, int m, int q_pos0, int topk, float* scores,
+                             int32_t* idx, void* ws, size_t ws_bytes,
+                             cslc_stream_t stream);
+
+/* The top-k stage alone, on given scores [B, L, Nc] fp32 (same selection rule
+ * and output layout as csa_indexer_topk; only the first n_vis(q_pos0+t)
+ * entries of row t are read). */
+cslc_status csa_topk(const float* scores, int B, int L, int Nc, int m, int q_pos0,
+                     int topk, int32_t* idx, cslc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* CSA core attention ("读完这篇…" §三 注意力计算: ordinary attention over the
+ * selected entries, KV shared by the heads)
+ *
+ *   o[b,t,h,:] = sum_{i in idx[b,t]} softmax_i(scale * q[b,t,h,:] . kv[b,i,:]) kv[b,i,:]
+ * with K = V = the compressed entry; slots holding -1 are skipped; a row with
+ * no valid slot outputs 0 and lse = -inf. fp32 accumulation, bf16 output.
+ *
+ *   q   [B, L, H, D] bf16    kv [B, Nc, D] bf16    idx [B, L, topk] int32
+ *   out [B, L, H, D] bf16    lse [B, L, H] fp32 natural-log sum-exp of the
+ *                            scaled logits, or NULL.
+ * Indices must lie in [-1, Nc); others are treated as -1.
+ */
+cslc_status csa_sparse_attn(const cslc_bf16* q, const cslc_bf16* kv, const int32_t* idx,
+                            int B, int L, int H, int D, int Nc, int topk, float scale,
+                            cslc_bf16* out, float* lse, cslc_stream_t stream);
+
+/* HCA core attention (first page §1.2: dense attention over all compressed
+ * entries), causal: query row t (absolute position q_pos0 + t) sees entries
+ * 0 .. n_vis-1 with n_vis = min(Nc, floor((q_pos0+t+1)/m')).
+ * Shapes as csa_sparse_attn without idx. */
+cslc_status hca_dense_attn(const cslc_bf16* q, const cslc_bf16* kv, int B, int L, int H,
+                           int D, int Nc, int m_prime, int q_pos0, float scale,
+                           cslc_bf16* out, float* lse, cslc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Mixed decode KV layout (first page §1.4 存储格式混)
+ *
+ * Splits entries kv [B, N, 128] bf16 into
+ *   nope  [B, N, 64] uint8  e4m3 codes of dims 0..63 divided by the entry scale
+ *   rope  [B, N, 64] bf16   dims 64..127 unchanged
+ *   scale [B, N] fp32       amax(|dims 0..63|) / 448 (1 when amax = 0)
+ * Scale and quotient are computed in fp32 (IEEE division); codes round to
+ * nearest even and saturate to +-448. 196 bytes per entry instead of 256.
+ */
+cslc_status cslc_quantize_kv_mixed(const cslc_bf16* kv, int B, int N, uint8_t* nope,
+                                   cslc_bf16* rope, float* scale, cslc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode: one new query token per sequence, all n_entries[b] entries visible.
+ *
+ * A CSA layer runs the indexer over the sequence's indexer keys, selects the
+ * top-k entries exactly (ties to the smaller index) and attends to them; an
+ * HCA layer attends densely to all entries. The KV is read in the mixed
+ * layout above and dequantised as e4m3 value * scale (rounded to bf16 for the
+ * tensor-core products).
+ */
+typedef struct {
+  int kind;                  /* 0 = CSA (indexer + top-k + sparse), 1 = HCA (dense) */
+  const cslc_bf16* q;        /* [B, H, 128] bf16 query heads */
+  const cslc_bf16* q_idx;    /* [B, H_I, 64] bf16 indexer query (CSA only) */
+  const cslc_bf16* w;        /* [B, H_I] bf16 indexer head weights (CSA only) */
+  const cslc_bf16* k_idx;    /* [B, n_max, 64] bf16 indexer keys (CSA only) */
+  const uint8_t* nope;       /* [B, n_max, 64] e4m3 */
+  const cslc_bf16* rope;     /* [B, n_max, 64] bf16 */
+  const float* kv_scale;     /* [B, n_max] fp32 */
+  const int32_t* n_entries;  /* [B] int32 device array, 0 <= n_entries[b] <= n_max */
+  int n_max;                 /* row stride (entries) of the per-sequence arrays */
+  int topk;                  /* CSA: entries kept per sequence, 1..2048 */
+  float scale;               /* softmax scale */
+  cslc_bf16* out;            /* [B, H, 128] bf16 */
+  int32_t* idx_out;          /* [B, topk] int32 selected entries (CSA), or NULL */
+  float* scores_out;         /* [B, n_max] fp32 indexer scores (CSA), or NULL */
+} cslc_decode_layer;
+
+/* Workspace for cslc_decode_step over these layers (the maximum over layers;
+ * layers run one after another on the stream and reuse it). */
+size_t cslc_decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers, int B,
+                                   int H, int HI);
+
+/* Runs the layers in order on `stream` (the hybrid C,H,C,H decode step is
+ * four layers). Requires D == 128, d_I == 64, H a multiple of 16 <= 128,
+ * 1 <= H_I <= 16. */
+cslc_status cslc_decode_step(const cslc_decode_layer* layers, int n_layers, int B, int H,
+                             int D, int HI, int dI, void* ws, size_t ws_bytes,
+                             cslc_stream_t stream);
+
+/* The decode top-k stage alone on given scores [B, n_max] fp32: idx [B, topk]
+ * = the min(topk, n_entries[b]) largest of the first n_entries[b] scores
+ * (ties to the smaller index), ascending, -1 padded. */
+size_t cslc_decode_topk_workspace_bytes(int B, int n_max, int topk);
+cslc_status cslc_decode_topk(const float* scores, const int32_t* n_entries, int B, int n_max,
+                             int topk, int32_t* idx, void* ws, size_t ws_bytes,
+                             cslc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSLC_H_ */

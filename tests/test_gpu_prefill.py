@@ -1,0 +1,298 @@
+"""GPU parity of the prefill path (compression, indexer + top-k, CSA sparse
+and HCA dense attention) against the CPU oracle, through the C ABI.
+
+Stage-isolated checks feed each kernel the oracle's own upstream values;
+end-to-end checks run the whole path from the raw inputs. Index sets are
+compared bit-exactly (top-k on given scores; and the indexer's selection is
+checked to be exactly the top-k of the scores it produced), floating-point
+outputs within max-abs 2e-2 / relative L2 1e-2.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from compressed_sparse_long_compress_b200 import workloads as W
+from tests.helpers import assert_close, assert_close_scaled, f64, rel_l2, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def C(cuda_device):
+    from compressed_sparse_long_compress_b200 import cslc
+    return cslc
+
+
+def dev(t):
+    return t.to("cuda:0")
+
+
+# --------------------------------------------------------------- compression
+
+@pytest.mark.parametrize("m,overlap,B,L", [
+    (4, True, 1, 4096), (4, True, 2, 4093), (4, True, 1, 3), (4, True, 1, 4), (2, True, 1, 130),
+    (128, False, 1, 4096), (128, False, 2, 4100), (128, False, 1, 100), (1, False, 1, 77), (8, False, 3, 999),
+])
+def test_compress_matches_oracle(C, m, overlap, B, L):
+    s = W.PrefillShape(B=B, L=L, H=16, m=m, overlap=overlap)
+    x = W.prefill_inputs(s, wid=11, with_indexer=False)
+    if overlap:
+        got = C.csa_compress(dev(x["c"]), dev(x["z"]), dev(x["pos_bias"]), m=m)
+    else:
+        got = C.hca_compress(dev(x["c"]), dev(x["z"]), dev(x["pos_bias"]), m_prime=m)
+    ref = O.compress(f64(x["c"]), f64(x["z"]), f64(x["pos_bias"]), m, overlap)
+    torch.cuda.synchronize()
+    assert got.shape == (B, L // m, 128)
+    if ref.size:
+        assert_close(f64(got), ref, what="compress")
+        assert np.mean(f64(got) == ref) > 0.98   # all but rounding-boundary cases bit-exact
+
+
+def test_compress_separate_prev_stream(C):
+    s = W.PrefillShape(B=2, L=1000, H=16, m=4)
+    x = W.prefill_inputs(s, wid=12, with_indexer=False, separate_prev_stream=True)
+    got = C.csa_compress(dev(x["c"]), dev(x["z"]), dev(x["pos_bias"]), m=4, c_b=dev(x["c_b"]), z_b=dev(x["z_b"]))
+    ref = O.compress(f64(x["c"]), f64(x["z"]), f64(x["pos_bias"]), 4, True, c_b=f64(x["c_b"]), z_b=f64(x["z_b"]))
+    assert_close(f64(got), ref, what="compress c_b/z_b")
+
+
+def test_compress_constant_and_identity(C):
+    c = torch.full((1, 512, 128), 0.375, dtype=torch.bfloat16)
+    z = W.randn_bf16((1, 512, 128), 5)
+    e = C.csa_compress(dev(c), dev(z), dev(W.randn_bf16((8, 128), 6, std=0.1)), m=4)
+    assert torch.all(e.cpu() == 0.375)
+    e1 = C.hca_compress(dev(z), dev(c), dev(torch.zeros(1, 128, dtype=torch.bfloat16)), m_prime=1)
+    assert torch.equal(e1.cpu(), z)
+
+
+# ------------------------------------------------------------------ mixed KV
+
+def test_quantize_kv_bitexact(C):
+    e = W.randn_bf16((3, 1000, 128), 21)
+    e[1, 5] = 0
+    e[2, 7, :64] = torch.tensor(1e-6).to(torch.bfloat16)
+    e[0, 9, 3] = 3e4
+    nope, rope, scale = C.quantize_kv_mixed(dev(e))
+    codes, rope_ref, scale_ref = O.quantize_kv_mixed(f64(e))
+    torch.cuda.synchronize()
+    assert np.array_equal(nope.cpu().numpy(), codes)
+    assert np.array_equal(scale.cpu().numpy(), scale_ref)
+    assert np.array_equal(f64(rope), rope_ref)
+
+
+# ----------------------------------------------------------- indexer + top-k
+
+def _indexer_case(C, B, L, HI, m, topk, q_pos0, wid, Nc=None):
+    s = W.PrefillShape(B=B, L=L, H=16, m=m, HI=HI, topk=topk)
+    x = W.prefill_inputs(s, wid=wid, with_indexer=True)
+    if Nc is not None:
+        x["k_idx"] = W.randn_bf16((B, Nc, 64), W.seed_of(wid, W.T_KIDX))
+    qi, w, k = dev(x["q_idx"]), dev(x["w"]), dev(x["k_idx"])
+    idx, scores = C.csa_indexer_topk(qi, w, k, m=m, topk=topk, q_pos0=q_pos0, scores=True)
+    idx_blocked, _ = C.csa_indexer_topk(qi, w, k, m=m, topk=topk, q_pos0=q_pos0)
+    torch.cuda.synchronize()
+    return x, idx.cpu().numpy(), idx_blocked.cpu().numpy(), f64(scores)
+
+
+@pytest.mark.parametrize("B,L,HI,m,topk,q_pos0,Nc", [
+    (1, 4096, 4, 4, 128, 0, None),          # the tiny workload's CSA layer
+    (2, 1000, 8, 4, 64, 0, None),           # ragged entry count (250, not a tile multiple)
+    (1, 777, 16, 4, 100, 37, None),         # 16 indexer heads, query offset
+    (1, 512, 1, 2, 300, 0, None),           # k above most rows' visible counts
+    (1, 300, 8, 4, 2048, 4000, 1100),       # later queries of a longer sequence
+])
+def test_indexer_topk_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
+    x, idx, idx_blocked, sc = _indexer_case(C, B, L, HI, m, topk, q_pos0, 31, Nc)
+    n_c = x["k_idx"].shape[1]
+    ref_s = O.indexer_scores(f64(x["q_idx"]), f64(x["w"]), f64(x["k_idx"]), m, q_pos0)
+    vis = np.isfinite(ref_s)
+    assert_close_scaled(np.where(vis, sc, -np.inf), ref_s, what="indexer scores")
+    # the selection is exactly the top-k of the scores the kernel produced
+    ref_on_gpu_scores = O.topk_select(np.where(vis, sc, -np.inf), m, topk, q_pos0)
+    assert np.array_equal(idx, ref_on_gpu_scores)
+    assert np.array_equal(idx, idx_blocked)
+    # and agrees with the oracle's own end-to-end selection up to near-ties
+    ref_idx = O.topk_select(ref_s, m, topk, q_pos0)
+    same = np.mean([np.array_equal(idx[b, t], ref_idx[b, t]) for b in range(B) for t in range(L)])
+    assert same > 0.97
+    # bit-exact visibility: count of valid slots is min(k, n_vis) and all < n_vis
+    for t in range(L):
+        nv = O.n_visible(q_pos0 + t, m, n_c)
+        v = idx[:, t][idx[:, t] >= 0].reshape(B, -1) if nv else np.zeros((B, 0))
+        assert (idx[:, t] >= 0).sum(axis=1).tolist() == [min(topk, nv)] * B
+        assert np.all(v < nv)
+
+
+@pytest.mark.parametrize("Nc,L,topk,q_pos0,ties", [
+    (1024, 4096, 128, 0, False), (16384, 300, 1024, 65000, False), (16384, 64, 2048, 65300, True),
+    (1000, 333, 1, 3000, True), (5000, 100, 1024, 19000, True),
+])
+def test_topk_on_given_scores_bitexact(C, Nc, L, topk, q_pos0, ties):
+    m = 4
+    s = W.rand_f32((1, L, Nc), seed=700 + Nc)
+    if ties:   # few distinct values: many exact ties at the threshold
+        s = torch.round(s * 2) / 2
+    idx = C.csa_topk(dev(s), m=m, topk=topk, q_pos0=q_pos0)
+    ref = O.topk_select(f64(s), m, topk, q_pos0)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_all_equal_scores(C):
+    s = torch.zeros(1, 40, 16384)
+    idx = C.csa_topk(dev(s), m=4, topk=1024, q_pos0=65000).cpu().numpy()
+    assert np.array_equal(idx[0], np.tile(np.arange(1024, dtype=np.int32), (40, 1)))
+    s = torch.full((1, 3, 16384), -1.5)
+    s[0, :, 7] = float("-inf")
+    idx = C.csa_topk(dev(s), m=4, topk=5, q_pos0=65000).cpu().numpy()
+    assert idx[0, 0].tolist() == [0, 1, 2, 3, 4]
+
+
+# ----------------------------------------------------------------- attention
+
+def _random_idx(rng, L, n_c, topk, holes=False):
+    idx = np.full((1, L, topk), -1, dtype=np.int32)
+    for t in range(L):
+        cnt = int(rng.integers(0, min(topk, n_c) + 1)) if t % 7 else min(topk, n_c)
+        sel = np.sort(rng.choice(n_c, cnt, replace=False)).astype(np.int32)
+        idx[0, t, :cnt] = sel
+        if holes and cnt > 4:
+            idx[0, t, 1] = -1
+            idx[0, t, 3] = n_c + 5      # out of range: treated as empty
+    return idx
+
+
+@pytest.mark.parametrize("H,L,n_c,topk,holes,q_scale", [
+    (16, 512, 1024, 128, False, 1.0), (64, 128, 16384, 1024, False, 1.0), (128, 64, 3000, 200, True, 1.0),
+    (64, 96, 2000, 1000, True, 8.0), (16, 40, 10, 2048, False, 1.0),
+])
+def test_sparse_attention_isolated(C, H, L, n_c, topk, holes, q_scale):
+    rng = np.random.default_rng(H + L)
+    q = W.randn_bf16((1, L, H, 128), 41)
+    if q_scale != 1.0:
+        q = (q.float() * q_scale).to(torch.bfloat16)
+    e = W.randn_bf16((1, n_c, 128), 42, std=0.4)
+    idx = _random_idx(rng, L, n_c, topk, holes)
+    scale = 1 / math.sqrt(128)
+    out, lse = C.csa_sparse_attn(dev(q), dev(e), dev(torch.from_numpy(idx)), scale, lse=True)
+    idx_ref = np.where((idx >= 0) & (idx < n_c), idx, -1)
+    o_ref, l_ref = O.sparse_attention(f64(q), f64(e), idx_ref, scale)
+    assert_close(f64(out), o_ref, what="sparse attn out")
+    assert_close(f64(lse), l_ref, what="sparse attn lse")
+
+
+@pytest.mark.parametrize("H,L,m,n_c,q_pos0,q_scale", [
+    (16, 4096, 128, 32, 0, 1.0), (64, 1001, 4, 250, 0, 1.0), (128, 300, 4, 2000, 5000, 1.0),
+    (64, 513, 128, 40, 4000, 8.0), (16, 50, 1, 50, 0, 1.0),
+])
+def test_dense_attention_isolated(C, H, L, m, n_c, q_pos0, q_scale):
+    q = W.randn_bf16((1, L, H, 128), 51)
+    if q_scale != 1.0:
+        q = (q.float() * q_scale).to(torch.bfloat16)
+    e = W.randn_bf16((1, n_c, 128), 52, std=0.4)
+    scale = 1 / math.sqrt(128)
+    out, lse = C.hca_dense_attn(dev(q), dev(e), m_prime=m, scale=scale, q_pos0=q_pos0, lse=True)
+    o_ref, l_ref = O.dense_causal_attention(f64(q), f64(e), m, scale, q_pos0)
+    assert_close(f64(out), o_ref, what="dense attn out")
+    assert_close(f64(lse), l_ref, what="dense attn lse")
+    # queries before the first complete window output exactly 0
+    for t in range(L):
+        if O.n_visible(q_pos0 + t, m, n_c) == 0:
+            assert np.all(f64(out)[0, t] == 0)
+
+
+def test_attention_runs_twice_identically(C):
+    q = dev(W.randn_bf16((1, 300, 64, 128), 61))
+    e = dev(W.randn_bf16((1, 2000, 128), 62))
+    a, _ = C.hca_dense_attn(q, e, m_prime=4, scale=0.088)
+    b, _ = C.hca_dense_attn(q, e, m_prime=4, scale=0.088)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- end to end
+
+def test_tiny_workload_end_to_end(C):
+    wl = W.WORKLOADS["tiny"]
+    s, sh = wl.csa, wl.hca
+    x = W.prefill_inputs(s, wl.wid)
+    xh = {"c": x["c"], "z": x["z"], "pos_bias": W.randn_bf16((sh.m, 128), W.seed_of(wl.wid, W.T_HBIAS), std=0.1)}
+    scale = s.scale
+    # GPU
+    e = C.csa_compress(dev(x["c"]), dev(x["z"]), dev(x["pos_bias"]), m=s.m)
+    idx, _ = C.csa_indexer_topk(dev(x["q_idx"]), dev(x["w"]), dev(x["k_idx"]), m=s.m, topk=s.topk)
+    o_csa, _ = C.csa_sparse_attn(dev(x["q"]), e, idx, scale)
+    eh = C.hca_compress(dev(xh["c"]), dev(xh["z"]), dev(xh["pos_bias"]), m_prime=sh.m)
+    o_hca, _ = C.hca_dense_attn(dev(x["q"]), eh, m_prime=sh.m, scale=scale)
+    torch.cuda.synchronize()
+    # oracle
+    e_ref = O.compress(f64(x["c"]), f64(x["z"]), f64(x["pos_bias"]), s.m, True)
+    s_ref = O.indexer_scores(f64(x["q_idx"]), f64(x["w"]), f64(x["k_idx"]), s.m)
+    idx_ref = O.topk_select(s_ref, s.m, s.topk)
+    o_ref, _ = O.sparse_attention(f64(x["q"]), e_ref, idx_ref, scale)
+    eh_ref = O.compress(f64(xh["c"]), f64(xh["z"]), f64(xh["pos_bias"]), sh.m, False)
+    oh_ref, _ = O.dense_causal_attention(f64(x["q"]), eh_ref, sh.m, scale)
+    assert_close(f64(e), e_ref, what="csa entries")
+    assert_close(f64(eh), eh_ref, what="hca entries")
+    idx = idx.cpu().numpy()
+    same = np.array([np.array_equal(idx[0, t], idx_ref[0, t]) for t in range(s.L)])
+    assert same.mean() > 0.97
+    assert_close(f64(o_csa)[:, same], o_ref[:, same], what="csa out (rows with identical selection)")
+    assert_close(f64(o_hca), oh_ref, what="hca out")
+    assert np.all(f64(o_csa)[0, : s.m - 1] == 0) and np.all(f64(o_hca)[0, : sh.m - 1] == 0)
+
+
+# -------------------------------------------------- full-size workloads (sampled)
+
+def test_csa_prefill_full_size_sampled(C):
+    wl = W.WORKLOADS["csa_prefill"]
+    s = wl.csa
+    x = W.prefill_inputs(s, wl.wid, device="cuda:0")
+    e = C.csa_compress(x["c"], x["z"], x["pos_bias"], m=s.m)
+    idx, _ = C.csa_indexer_topk(x["q_idx"], x["w"], x["k_idx"], m=s.m, topk=s.topk)
+    out, _ = C.csa_sparse_attn(x["q"], e, idx, s.scale)
+    idx_s, scores = C.csa_indexer_topk(x["q_idx"], x["w"], x["k_idx"], m=s.m, topk=s.topk, scores=True)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_s)
+    rows = sample_rows(s.L, 48, seed=2001)
+    e_ref = O.compress(f64(x["c"]), f64(x["z"]), f64(x["pos_bias"]), s.m, True)
+    assert_close(f64(e), e_ref, what="entries")
+    qi, ww = f64(x["q_idx"]), f64(x["w"])
+    s_ref = np.full((1, len(rows), s.n_c), -np.inf)
+    k_all = f64(x["k_idx"])
+    for r, t in enumerate(rows):
+        s_ref[:, r] = O.indexer_scores(qi[:, t:t + 1], ww[:, t:t + 1], k_all, s.m, q_pos0=int(t))[:, 0]
+    sc = f64(scores[:, torch.as_tensor(rows, device=scores.device)])
+    vis = np.isfinite(s_ref)
+    assert_close_scaled(np.where(vis, sc, -np.inf), s_ref, what="scores")
+    g_idx = idx[:, torch.as_tensor(rows, device=idx.device)].cpu().numpy()
+    for r, t in enumerate(rows):
+        assert np.array_equal(g_idx[0, r], O.topk_select_row(sc[0, r], O.n_visible(int(t), s.m, s.n_c), s.topk))
+    ref_idx = np.stack([O.topk_select_row(s_ref[0, r], O.n_visible(int(t), s.m, s.n_c), s.topk)
+                        for r, t in enumerate(rows)])[None]
+    same = np.array([np.array_equal(g_idx[0, r], ref_idx[0, r]) for r in range(len(rows))])
+    assert same.mean() > 0.9
+    q_rows = f64(x["q"][:, torch.as_tensor(rows, device=x["q"].device)])
+    o_ref, _ = O.sparse_attention(q_rows, e_ref, ref_idx, s.scale)
+    o_got = f64(out[:, torch.as_tensor(rows, device=out.device)])
+    assert_close(o_got[:, same], o_ref[:, same], what="csa out")
+
+
+def test_hca_prefill_full_size_sampled(C):
+    wl = W.WORKLOADS["hca_prefill"]
+    s = wl.hca
+    x = W.prefill_inputs(s, wl.wid, device="cuda:0", with_indexer=False)
+    e = C.hca_compress(x["c"], x["z"], x["pos_bias"], m_prime=s.m)
+    out, _ = C.hca_dense_attn(x["q"], e, m_prime=s.m, scale=s.scale)
+    torch.cuda.synchronize()
+    e_ref = O.compress(f64(x["c"]), f64(x["z"]), f64(x["pos_bias"]), s.m, False)
+    assert_close(f64(e), e_ref, what="entries")
+    rows = sample_rows(s.L, 64, seed=3001)
+    rows_t = torch.as_tensor(rows, device=x["q"].device)
+    q_rows = f64(x["q"][:, rows_t])
+    o_ref = np.zeros_like(q_rows)
+    for r, t in enumerate(rows):
+        o_ref[:, r:r + 1], _ = O.dense_causal_attention(q_rows[:, r:r + 1], e_ref, s.m, s.scale, q_pos0=int(t))
+    assert_close(f64(out[:, rows_t]), o_ref, what="hca out")
