@@ -37,6 +37,7 @@ cslc_status launch_sparse_attn(const uint16_t*, const uint16_t*, const int32_t*,
 cslc_status launch_dense_attn(const uint16_t*, const uint16_t*, int, int, int, int, int, int, float,
                               uint16_t*, float*, cudaStream_t);
 size_t decode_workspace_bytes(const cslc_decode_layer*, int, int, int);
+int sparse_attn_sm100_read_error();
 size_t decode_topk_workspace_bytes(int, int, int);
 cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*, size_t, cudaStream_t);
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
@@ -80,6 +81,9 @@ const char* cslc_last_error(void) { return g_err; }
 cslc_status cslc_sync_status(cslc_stream_t stream) {
   const cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "cslc_sync_status: %s", cudaGetErrorString(e));
+  const int code = sparse_attn_sm100_read_error();
+  if (code != 0)
+    return set_error(CSLC_ERR_DEVICE_CHECK, "csa_sparse_attn: a pipeline wait timed out (code %d)", code);
   return CSLC_OK;
 }
 

@@ -247,10 +247,17 @@ static void attn_configure() {
   }
 }
 
+bool sparse_attn_sm100_supported(int H);
+cslc_status launch_sparse_attn_sm100(const uint16_t*, const uint16_t*, const int32_t*, int, int, int, int, int,
+                                     float, uint16_t*, float*, cudaStream_t);
+
 cslc_status launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int L,
                                int H, int Nc, int topk, float scale, uint16_t* out, float* lse,
                                cudaStream_t stream) {
   if (B == 0 || L == 0) return CSLC_OK;
+  // tcgen05 kernel for up to 64 heads; more heads take the warp-level MMA kernel below
+  if (sparse_attn_sm100_supported(H))
+    return launch_sparse_attn_sm100(q, kv, idx, B, L, H, Nc, topk, scale, out, lse, stream);
   attn_configure<true, 1>();
   dim3 grid(L, B);
   attention_kernel<true, 1><<<grid, (H / 16) * 32, attn_smem<true, 1>(H, topk), stream>>>(

@@ -619,6 +619,15 @@ static cslc_status run_attention(const cslc_decode_layer& l, int B, int H, const
                                  DecodeWs& w, cudaStream_t stream) {
   const int splits = layer_splits(l);
   const size_t smem = (size_t)H * 256 + DTILE * 256;
+  static int configured_for = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_for != dev) {
+    const int max_smem = 128 * 256 + DTILE * 256;
+    cudaFuncSetAttribute(decode_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    cudaFuncSetAttribute(decode_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    configured_for = dev;
+  }
   const dim3 grid(splits, B);
   const float sl2 = l.scale * kLog2e;
   if (l.kind == 0)

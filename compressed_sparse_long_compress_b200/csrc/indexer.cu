@@ -4,7 +4,7 @@
 // V3.2 DSA indexer):
 //   S[t, i] = sum_h w[t, h] * max(0, q_I[t, h, :] . k_I[i, :])
 //
-// CTA = 64 query rows (4 warps x 16 rows) and all H_I heads. The CTA's
+// CTA = 64 query rows (4 warps x 16 rows) x up to 1024 entries, all H_I heads. The CTA's
 // queries (64 rows x H_I heads x 64 dims, bf16) stay in shared memory; key
 // tiles of 64 entries x 64 dims stream through a two-stage cp.async ring. Per
 // key tile each warp keeps the tile's B fragments in registers and runs, for
@@ -20,6 +20,7 @@ namespace cslc {
 constexpr int IDX_ROWS = 64;     // query rows per CTA
 constexpr int IDX_TILE = 64;     // entries per key tile
 constexpr int IDX_THREADS = 128;
+constexpr int IDX_SPLIT_TILES = 16;   // key tiles (1024 entries) per CTA
 
 __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
     const uint16_t* __restrict__ q_idx, const uint16_t* __restrict__ w,
@@ -31,14 +32,20 @@ __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
   float* w_s = reinterpret_cast<float*>(k_s + 2 * IDX_TILE * 128);   // [64 rows][HI]
 
   const int b = blockIdx.y;
-  const int nblk = gridDim.x;
-  const int r0 = row_begin + (nblk - 1 - blockIdx.x) * IDX_ROWS;   // heavy (late) rows first
+  // blockIdx.x enumerates (entry split, row block); row blocks run heavy (late) rows first
+  const int n_rb = (row_end - row_begin + IDX_ROWS - 1) / IDX_ROWS;
+  const int rblk = n_rb - 1 - (int)(blockIdx.x % n_rb);
+  const int split = (int)(blockIdx.x / n_rb);
+  const int r0 = row_begin + rblk * IDX_ROWS;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
 
   const int last_row = min(r0 + IDX_ROWS, row_end) - 1;
   const int nv_max = n_visible((long long)q_pos0 + last_row, m, Nc);
-  const int n_tiles = (nv_max + IDX_TILE - 1) / IDX_TILE;
+  const int tile_lo = split * IDX_SPLIT_TILES;
+  const int tile_hi = min((nv_max + IDX_TILE - 1) / IDX_TILE, tile_lo + IDX_SPLIT_TILES);
+  if (tile_lo >= tile_hi) return;   // uniform: this split holds no visible entry of the block
+  const int n_tiles = tile_hi - tile_lo;
 
   // queries -> smem (16-byte chunks, swizzled per 128-byte row)
   for (int x = tid; x < HI * IDX_ROWS * 8; x += IDX_THREADS) {
@@ -54,7 +61,7 @@ __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
     w_s[x] = r < row_end ? bf16_to_f(w[((size_t)b * L + r) * HI + h]) : 0.f;
   }
   auto load_tile = [&](int tile, int stage) {
-    const int e0 = tile * IDX_TILE;
+    const int e0 = (tile_lo + tile) * IDX_TILE;
     for (int x = tid; x < IDX_TILE * 8; x += IDX_THREADS) {
       const int chunk = x & 7, row = x >> 3;
       const int e = e0 + row;
@@ -81,7 +88,7 @@ __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
     cp_async_wait<1>();
     __syncthreads();
 
-    const int e0 = tile * IDX_TILE;
+    const int e0 = (tile_lo + tile) * IDX_TILE;
     if (e0 < warp_nv_max) {
       // B fragments of the key tile: b[nt][ks][2] for 8 n-tiles of 8 entries and 4 k-steps
       uint32_t bf[8][4][2];
@@ -170,7 +177,11 @@ cslc_status launch_indexer_scores(const uint16_t* q_idx, const uint16_t* w, cons
                          (int)indexer_smem_bytes(16));
     configured_for = dev;
   }
-  dim3 grid((row_end - row_begin + IDX_ROWS - 1) / IDX_ROWS, B);
+  const int n_rb = (row_end - row_begin + IDX_ROWS - 1) / IDX_ROWS;
+  const int nv_max = n_visible((long long)q_pos0 + row_end - 1, m, Nc);
+  const int n_split = ((nv_max + IDX_TILE - 1) / IDX_TILE + IDX_SPLIT_TILES - 1) / IDX_SPLIT_TILES;
+  if (n_split == 0) return CSLC_OK;
+  dim3 grid(n_rb * n_split, B);
   indexer_scores_kernel<<<grid, IDX_THREADS, smem, stream>>>(q_idx, w, k_idx, L, Nc, HI, m, q_pos0,
                                                              row_begin, row_end, scores, rows_in_buf);
   return check_launch("indexer_scores_kernel");
