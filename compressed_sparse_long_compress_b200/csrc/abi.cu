@@ -43,7 +43,7 @@ cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*,
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
 
 constexpr int kMaxTopk = 2048;
-constexpr int kMaxPrefillTopkNc = 49152;   // row of keys must fit in shared memory
+constexpr int kMaxPrefillTopkNc = 49152;   // a row of scores must fit in shared memory
 
 static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -59,9 +59,10 @@ static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
   } while (0)
 
 // scores rows are processed in blocks of this many rows when the caller does
-// not keep them, so a block stays resident in L2 between the two kernels
+// not keep them: large enough that every indexer launch fills the GPU many
+// times over (the scores' HBM round trip costs far less than idle SMs)
 static int score_block_rows(int Nc) {
-  const long long budget = 48ll << 20;   // bytes of scores per block
+  const long long budget = 256ll << 20;   // bytes of scores per block
   long long rows = budget / ((long long)Nc * 4);
   rows = rows < 64 ? 64 : rows;
   rows = (rows / 64) * 64;

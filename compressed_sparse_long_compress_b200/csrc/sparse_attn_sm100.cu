@@ -6,25 +6,30 @@
 //
 // Formulation (per query token t, entries gathered in tiles of 128):
 //   S^T[e, h] = E[e, :] . Q_t[h, :]          (M = 128 entries, N = H heads, K = 128)
-//   P^T[e, h] = exp2(scale*log2e*S^T - m[h]) (softmax over e, per head h)
+//   P^T[e, h] = 2^(c*S^T[e,h] - m[h])        (c = scale*log2 e; softmax over e per head)
 //   O^T[d, h] += sum_e E[e, d] P^T[e, h]      (M = 128 dims, N = 64, K = 128 entries)
 // Putting the 128 gathered entries on the MMA's M side keeps M = 128 (full
-// rate) although a token has only 64 heads, and lets both products read the
-// same shared-memory tile of entries (K-major for S^T, MN-major for O^T).
+// rate) although a token has only 64 heads, and both products read the same
+// shared-memory tile of entries (K-major for S^T, MN-major for O^T).
 //
 // CTA roles (persistent CTAs, one per SM, loop over tokens):
-//   warps 0-3  softmax + epilogue: thread = TMEM lane = entry of the tile; the
-//              per-head running max m[h] is shared by the CTA and only updated
-//              (exact tile max, O^T rescale) when a score exceeds it by more
-//              than 2^8 -- always on a token's first tile, rarely after; P^T
-//              rows go to swizzled shared memory; at the token's end the head
-//              sums are reduced, O^T is read from TMEM, normalised, transposed
-//              through shared memory and stored
-//   warps 4-6  producer: per token the index row and Q_t (cp.async), then the
-//              gathered entry tiles (cp.async, 16 B chunks, 128-byte swizzle)
-//              into a STAGES-deep ring
-//   warp 7     TMEM allocation and the single MMA-issuing thread
-// (8 warps = 2 per SM sub-partition, so each thread may use up to 255 registers)
+//   warps 0-7   softmax + epilogue. Warp w owns TMEM lane quadrant w & 3 (32
+//               entries of the tile, or 32 output dims) and head half w >> 2,
+//               so two warps share each SM sub-partition. The per-head
+//               running max m[h] is CTA-wide and only moved (exact tile max
+//               by warp reduction, O^T rescale in TMEM) on a token's first
+//               tile or when a probability would exceed 2^8 -- rare after the
+//               first tile. P^T rows go to 128-byte-swizzled shared memory.
+//               At the token's end the head sums are reduced (butterfly
+//               reduce-scatter), O^T is read from TMEM, normalised,
+//               transposed through shared memory and stored.
+//   warps 8-10  producer: per token the index row and Q_t (2-D TMA), then the
+//               gathered entry tiles (cp.async 16 B chunks, 128-byte swizzle;
+//               the copies arrive on the stage barrier as they land) into a
+//               STAGES-deep ring. (Measured on B200: random 256-byte rows from
+//               an L2-resident table gather at ~10 TB/s with cp.async but only
+//               ~2 TB/s with TMA tile::gather4.)
+//   warp 11     TMEM allocation and the single MMA-issuing thread.
 // TMEM: S^T double buffer (2 x 64 columns) + O^T double buffer (2 x 64).
 // Every wait is time-bounded; a timeout raises a CTA-wide abort, records an
 // error code in a device word read by cslc_sync_status, and all roles leave.
@@ -39,23 +44,28 @@ __device__ int g_sparse_attn_err = 0;
 
 namespace {
 
-constexpr int SA_THREADS = 256;
-constexpr int SA_NPROD = 96;             // producer threads (warps 4-6)
+constexpr int SA_THREADS = 384;
+constexpr int SA_NSOFT = 256;             // softmax threads (warps 0-7)
+constexpr int SA_PROD_WARP0 = 8;          // producer warps 8-10
+constexpr int SA_NPROD = 96;
+constexpr int SA_MMA_WARP = 11;
 constexpr int SA_TILE = 128;              // entries per tile (MMA M)
+constexpr int SA_ROWS_PER_PROD = (SA_TILE * 16 + SA_NPROD - 1) / SA_NPROD;   // 22 (6 rows per pass)
 constexpr int SA_NP = 64;                 // padded head count of P^T / O^T
 constexpr int SA_STAGES = 4;
 constexpr int SA_E_BYTES = SA_TILE * 256; // 32 KB per entry tile
 constexpr int SA_P_BYTES = SA_TILE * 128; // 16 KB per P^T tile (64 heads bf16)
 constexpr int SA_Q_BYTES = SA_NP * 256;   // 16 KB (also the output staging)
 constexpr int SA_MAXK = 2048;
+constexpr float SA_OVERFLOW = 256.f;      // probabilities up to 2^8 are kept unrescaled
 
-enum { ERR_KV_EMPTY = 1, ERR_TOK_FULL, ERR_KV_FULL, ERR_S_FREE, ERR_P_FULL, ERR_O_FREE, ERR_S_FULL,
+enum { ERR_KV_EMPTY = 1, ERR_TOK_FULL, ERR_KV_FULL, ERR_P_FULL, ERR_O_FREE, ERR_S_FULL,
        ERR_PV_DONE, ERR_O_FULL, ERR_Q_EMPTY, ERR_FINAL };
 
 struct __align__(8) SaBars {
   uint64_t kv_full[SA_STAGES], kv_empty[SA_STAGES];
   uint64_t tok_full[2], q_empty[2];
-  uint64_t s_full[2], s_free[2];
+  uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done;
   uint64_t o_full[2], o_free[2];
@@ -67,20 +77,61 @@ struct SaSmall {
   uint32_t tmem_base;
   int abort_flag;
   int n_tiles[2];
-  int max_slot[2];
+  int last_w[2][4];
   int any_rescale;
-  float mref[SA_NP];       // running max per head (log2 units)
-  float alpha[SA_NP];
-  float inv_l[SA_NP];
-  float red[4][SA_NP];     // per-warp partials
+  __align__(16) float mref[SA_NP];   // running max per head (log2 units of c*S)
+  __align__(16) float alpha[SA_NP];
+  __align__(16) float inv_l[SA_NP];
+  float red[4][SA_NP];               // per lane-quadrant partials
 };
+
+// Reduce-scatter of N per-lane values over the warp: returns, in every lane,
+// the warp sum of value index rs_index<N>(lane).
+template <int N, int OFF>
+struct ReduceScatter {
+  static __device__ __forceinline__ float run(const float* v, int lane) {
+    float w[N / 2];
+    const bool up = (lane & OFF) != 0;
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const float send = up ? v[i] : v[i + N / 2];
+      const float keep = up ? v[i + N / 2] : v[i];
+      w[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+    }
+    return ReduceScatter<N / 2, OFF / 2>::run(w, lane);
+  }
+};
+template <int OFF>
+struct ReduceScatter<1, OFF> {
+  static __device__ __forceinline__ float run(const float* v, int) {
+    float x = v[0];
+#pragma unroll
+    for (int o = OFF; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+  }
+};
+template <int N>
+__device__ __forceinline__ int rs_index(int lane) {
+  int idx = 0, n = N;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      if (lane & off) idx += n / 2;
+      n >>= 1;
+    }
+  }
+  return idx;
+}
 
 }  // namespace
 
 template <int H>
 __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ kv, const int32_t* __restrict__ idx,
-    int B, int L, int Nc, int topk, float scale_log2, uint16_t* __restrict__ out, float* __restrict__ lse) {
+    int B, int L, int Nc, int topk, float scale_log2, uint16_t* __restrict__ out, float* __restrict__ lse,
+    const __grid_constant__ CUtensorMap tm_q) {
+  constexpr int HT = H / 2;           // heads per softmax thread
+  static_assert(HT % 8 == 0 && HT <= 32, "H must be 16, 32 or 64");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* e_s = smem;                                       // [STAGES][2 kb][128][128 B]
@@ -96,17 +147,17 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
   if (tid == 0) {
     for (int s = 0; s < SA_STAGES; ++s) { mbar_init(&bars.kv_full[s], SA_NPROD); mbar_init(&bars.kv_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.tok_full[i], SA_NPROD); mbar_init(&bars.q_empty[i], 128);
-      mbar_init(&bars.s_full[i], 1); mbar_init(&bars.s_free[i], 128);
-      mbar_init(&bars.p_full[i], 128);
-      mbar_init(&bars.o_full[i], 1); mbar_init(&bars.o_free[i], 128);
+      mbar_init(&bars.tok_full[i], 1); mbar_init(&bars.q_empty[i], SA_NSOFT);
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.p_full[i], SA_NSOFT);
+      mbar_init(&bars.o_full[i], 1); mbar_init(&bars.o_free[i], SA_NSOFT);
     }
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.final_bar, 1);
     sm->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == 7) tmem_alloc(&sm->tmem_base, 256);
+  if (warp == SA_MMA_WARP) tmem_alloc(&sm->tmem_base, 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -114,12 +165,18 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
   volatile int* abortp = &sm->abort_flag;
   int* errp = &g_sparse_attn_err;
 
-  if (warp >= 4 && warp < 7) {
+  if (warp >= SA_PROD_WARP0 && warp < SA_MMA_WARP) {
     // ------------------------------------------------------------ producer
-    const int p = tid - 128;           // 0..95
+    // Three warps. Per token: the index row (plain loads) and Q_t (2-D TMA,
+    // completing on tok_full); per tile: 128 gathered rows x 16 chunks of
+    // 16 B with cp.async into the 128-byte swizzled layout. Each thread's
+    // copies arrive on the stage's barrier when they land (no waiting here).
+    const int p = tid - SA_PROD_WARP0 * 32;   // 0..95
+    const int pc = p & 15, pr0 = p >> 4;      // 16-byte column and first row of this thread
     int kv_it = 0;
     bool ok = true;
     long long tk = 0;
+    if (p == 0) tma_prefetch_map(&tm_q);
     for (long long g = blockIdx.x; g < n_tok && ok; g += gridDim.x, ++tk) {
       const int qb = (int)(tk & 1);
       if (tk >= 2) {
@@ -128,7 +185,6 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         ok = !named_bar_or(1, SA_NPROD, !w);
         if (!ok) break;
       }
-      // index row -> smem, last valid slot
       const int32_t* irow = idx + g * (long long)topk;
       int32_t* is = idx_s + qb * SA_MAXK;
       int last = 0;
@@ -139,26 +195,17 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         if (e >= 0) last = s + 1;
       }
       last = __reduce_max_sync(0xffffffffu, last);
-      if (p == 0) sm->max_slot[qb] = 0;
+      if (lane == 0) sm->last_w[qb][p >> 5] = last;
       named_bar(1, SA_NPROD);
-      if (lane == 0) atomicMax(&sm->max_slot[qb], last);
-      // Q_t: H rows x 256 B -> [2 kb][64][128 B] (rows >= H stay unused)
-      uint8_t* qd = q_s + qb * SA_Q_BYTES;
-      const uint16_t* qsrc = q + g * (long long)H * kD;
-      for (int x = p; x < H * 16; x += SA_NPROD) {
-        const int r = x >> 4, c = x & 15;
-        cp_async16(smem_u32(qd + (c >> 3) * (SA_NP * 128) + sw128(r, c & 7)), qsrc + r * kD + c * 8, true);
+      const int nt = (max(max(sm->last_w[qb][0], sm->last_w[qb][1]), sm->last_w[qb][2]) + SA_TILE - 1) / SA_TILE;
+      if (p == 0) {
+        sm->n_tiles[qb] = nt;
+        uint8_t* qd = q_s + qb * SA_Q_BYTES;
+        mbar_arrive_expect_tx(&bars.tok_full[qb], (uint32_t)(H * 256));
+        tma_load_2d(qd, &tm_q, 0, (int)(g * H), &bars.tok_full[qb]);
+        tma_load_2d(qd + SA_NP * 128, &tm_q, 64, (int)(g * H), &bars.tok_full[qb]);
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      named_bar(1, SA_NPROD);
-      const int nt = (sm->max_slot[qb] + SA_TILE - 1) / SA_TILE;
-      if (p == 0) sm->n_tiles[qb] = nt;
-      mbar_arrive(&bars.tok_full[qb]);
-      // entry tiles: 128 rows x 16 chunks of 16 B, chunk x -> row x >> 4, chunk x & 15
       const uint16_t* kvb = kv + (g / L) * (long long)Nc * kD;
-      int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int stage = kv_it % SA_STAGES;
         if (kv_it >= SA_STAGES) {
@@ -167,141 +214,153 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
           ok = !named_bar_or(1, SA_NPROD, !w);
           if (!ok) break;
         }
-        uint8_t* ed = e_s + stage * SA_E_BYTES;
-        for (int x = p; x < SA_TILE * 16; x += SA_NPROD) {
-          const int r = x >> 4, c = x & 15;
+        // this thread always copies 16-byte column pc of rows pr0 + 6 i
+        const uint32_t ed = smem_u32(e_s + stage * SA_E_BYTES) + (pc >> 3) * (SA_TILE * 128);
+        int ev[SA_ROWS_PER_PROD];
+#pragma unroll
+        for (int i = 0; i < SA_ROWS_PER_PROD; ++i) {
+          const int r = pr0 + 6 * i;
           const int slot = j * SA_TILE + r;
-          const int e = slot < topk ? is[slot] : -1;
-          cp_async16(smem_u32(ed + (c >> 3) * (SA_TILE * 128) + sw128(r, c & 7)),
-                     kvb + (long long)(e < 0 ? 0 : e) * kD + c * 8, e >= 0);
+          ev[i] = (r < SA_TILE && slot < topk) ? is[slot] : -1;
         }
-        cp_async_commit();
-        ++issued;
-        if (issued >= SA_STAGES - 1) {
-          cp_async_wait<SA_STAGES - 2>();
-          fence_proxy_async_smem();
-          mbar_arrive(&bars.kv_full[(kv_it - (SA_STAGES - 2)) % SA_STAGES]);
-          --issued;
+#pragma unroll
+        for (int i = 0; i < SA_ROWS_PER_PROD; ++i) {
+          const int r = pr0 + 6 * i;
+          if (r < SA_TILE)
+            cp_async16(ed + sw128(r, pc & 7), kvb + (long long)(ev[i] < 0 ? 0 : ev[i]) * kD + pc * 8, ev[i] >= 0);
         }
+        cp_async_mbar_arrive(&bars.kv_full[stage]);
         ++kv_it;
       }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      for (int k = issued; k > 0; --k) mbar_arrive(&bars.kv_full[(kv_it - k) % SA_STAGES]);
     }
     cp_async_wait<0>();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------ softmax + epilogue
-    const int s_lane = tid;                // 0..127 = TMEM lane = entry row / output dim
-    const int wq = warp;                   // TMEM lane quadrant
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int q4 = warp & 3, hh = warp >> 2;
+    const int row = q4 * 32 + lane;         // TMEM lane = entry row of the tile / output dim
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const int h0 = hh * HT;                 // first head of this thread
     int s_it = 0, p_it = 0;
     bool ok = true;
     long long tk = 0;
     for (long long g = blockIdx.x; g < n_tok && ok; g += gridDim.x, ++tk) {
       const int qb = (int)(tk & 1), ob = qb;
-      bool w = true;
-      if (s_lane == 0) w = mbar_wait(&bars.tok_full[qb], (uint32_t)((tk >> 1) & 1), abortp, errp, ERR_TOK_FULL);
-      ok = !named_bar_or(2, 128, !w);
-      const int nt = sm->n_tiles[qb];
-      if (s_lane < SA_NP) sm->mref[s_lane] = -INFINITY;
-      named_bar(2, 128);
+      {
+        bool w = true;
+        if (tid == 0) w = mbar_wait(&bars.tok_full[qb], (uint32_t)((tk >> 1) & 1), abortp, errp, ERR_TOK_FULL);
+        ok = !named_bar_or(2, SA_NSOFT, !w);
+      }
       if (!ok) break;
+      const int nt = sm->n_tiles[qb];
+      if (tid < SA_NP) sm->mref[tid] = -INFINITY;
+      named_bar(2, SA_NSOFT);
       const int32_t* is = idx_s + qb * SA_MAXK;
-      float lpart[H];
+      float lpart[HT];
 #pragma unroll
-      for (int h = 0; h < H; ++h) lpart[h] = 0.f;
+      for (int h = 0; h < HT; ++h) lpart[h] = 0.f;
 
       for (int j = 0; j < nt; ++j) {
         const int sb = s_it & 1, pb = p_it & 1;
-        bool w = true;
-        if (s_lane == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
-        ok = !named_bar_or(2, 128, !w);
+        {
+          bool w = true;
+          if (tid == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
+          ok = !named_bar_or(2, SA_NSOFT, !w);
+        }
         if (!ok) break;
         tc_fence_after();
-        float sv[H];
+        float raw[HT];
         {
           uint32_t r[32];
+          tmem_ld32(tmem + lane_off + sb * 64 + h0, r);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c0 = 0; c0 < H; c0 += 32) {
-            tmem_ld32(tmem + lane_off + sb * 64 + c0, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (c0 + k < H) sv[c0 + k] = __uint_as_float(r[k]);
-          }
+          for (int h = 0; h < HT; ++h) raw[h] = __uint_as_float(r[h]);
         }
-        tc_fence_before();
-        mbar_arrive(&bars.s_free[sb]);
-        const int slot = j * SA_TILE + s_lane;
+        const int slot = j * SA_TILE + row;
         const bool valid = slot < topk && is[slot] >= 0;
-        bool exceed = false;
+        float pr[HT];
+        bool slow = (j == 0);
+        if (!slow) {
+          float pmax = 0.f;
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-          sv[h] = valid ? sv[h] * scale_log2 : -INFINITY;
-          exceed |= sv[h] > sm->mref[h] + 8.f;
-        }
-        if (j == 0 || named_bar_or(3, 128, exceed)) {
-          // exact per-head maximum of this tile, then the new running max
+          for (int h4 = 0; h4 < HT; h4 += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(&sm->mref[h0 + h4]);
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-          for (int h = 0; h < H; ++h) {
-            const float mx = warp_max(sv[h]);
-            if (lane == 0) sm->red[wq][h] = mx;
+            for (int k = 0; k < 4; ++k) {
+              pr[h4 + k] = valid ? ex2_approx(fmaf(raw[h4 + k], scale_log2, -mm[k])) : 0.f;
+              pmax = fmaxf(pmax, pr[h4 + k]);
+            }
           }
-          if (s_lane == 0) sm->any_rescale = 0;
-          named_bar(2, 128);
-          if (s_lane < H) {
-            const float old = sm->mref[s_lane];
-            const float tmx = fmaxf(fmaxf(sm->red[0][s_lane], sm->red[1][s_lane]), fmaxf(sm->red[2][s_lane], sm->red[3][s_lane]));
+          slow = named_bar_or(3, SA_NSOFT, pmax > SA_OVERFLOW);
+        }
+        if (slow) {
+          // exact per-head maximum of this tile (raw scores; scaled below)
+#pragma unroll
+          for (int h = 0; h < HT; ++h) {
+            const float mx = warp_redux_max(valid ? raw[h] : -INFINITY);
+            if (lane == 0) sm->red[q4][h0 + h] = mx;
+          }
+          if (tid == 0) sm->any_rescale = 0;
+          named_bar(2, SA_NSOFT);
+          if (tid < H) {
+            const float old = sm->mref[tid];
+            const float tmx = fmaxf(fmaxf(sm->red[0][tid], sm->red[1][tid]), fmaxf(sm->red[2][tid], sm->red[3][tid])) * scale_log2;
             const float nm = fmaxf(old, tmx);
             float a = 1.f;
-            if (old != -INFINITY && nm != old) a = exp2f(old - nm);
-            else if (old == -INFINITY) a = 0.f;
-            sm->alpha[s_lane] = a;
-            sm->mref[s_lane] = nm;
+            if (old == -INFINITY) a = 0.f;
+            else if (nm != old) a = ex2_approx(old - nm);
+            sm->alpha[tid] = a;
+            sm->mref[tid] = nm;
             if (a != 1.f && j > 0) sm->any_rescale = 1;
+          } else if (tid < SA_NP) {
+            sm->alpha[tid] = 1.f;
           }
-          named_bar(2, 128);
+          named_bar(2, SA_NSOFT);
 #pragma unroll
-          for (int h = 0; h < H; ++h) lpart[h] *= sm->alpha[h];
+          for (int h = 0; h < HT; ++h) lpart[h] *= sm->alpha[h0 + h];
           if (sm->any_rescale) {
             // O^T must be stable: the previous tile's PV has to be complete
-            bool w2 = true;
-            if (s_lane == 0) w2 = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
-            ok = !named_bar_or(2, 128, !w2);
+            {
+              bool w = true;
+              if (tid == 0) w = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
+              ok = !named_bar_or(2, SA_NSOFT, !w);
+            }
             if (!ok) break;
             tc_fence_after();
             uint32_t r[32];
+            const uint32_t oc = tmem + lane_off + 128 + ob * 64 + hh * 32;
+            tmem_ld32(oc, r);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c0 = 0; c0 < SA_NP; c0 += 32) {
-              tmem_ld32(tmem + lane_off + 128 + ob * 64 + c0, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * (c0 + k < H ? sm->alpha[c0 + k] : 1.f));
-              tmem_st32(tmem + lane_off + 128 + ob * 64 + c0, r);
-            }
+            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * sm->alpha[hh * 32 + k]);
+            tmem_st32(oc, r);
             tmem_wait_st();
           }
-        }
-        // P^T row of this entry: 64 bf16 (heads >= H are zero)
-        uint32_t pk[SA_NP / 2];
 #pragma unroll
-        for (int h2 = 0; h2 < SA_NP / 2; ++h2) {
-          float a = 0.f, b = 0.f;
-          if (2 * h2 < H) {
-            const float m0 = sm->mref[2 * h2], m1 = sm->mref[2 * h2 + 1];
-            a = valid ? exp2f(sv[2 * h2] - m0) : 0.f;
-            b = valid ? exp2f(sv[2 * h2 + 1] - m1) : 0.f;
-            lpart[2 * h2] += a;
-            lpart[2 * h2 + 1] += b;
+          for (int h4 = 0; h4 < HT; h4 += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(&sm->mref[h0 + h4]);
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              pr[h4 + k] = valid ? ex2_approx(fmaf(raw[h4 + k], scale_log2, -mm[k])) : 0.f;
           }
-          pk[h2] = pack_bf16x2(a, b);
         }
+#pragma unroll
+        for (int h = 0; h < HT; ++h) lpart[h] += pr[h];
+        // P^T row: this thread's heads h0 .. h0+HT-1 (chunks of 8 heads); the
+        // second head half also zero-fills the padding heads H .. 63
         uint8_t* prow = p_s + pb * SA_P_BYTES;
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          *reinterpret_cast<uint4*>(prow + sw128(s_lane, c8)) =
-              make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        for (int c8 = 0; c8 < HT / 8; ++c8) {
+          const uint4 v = make_uint4(pack_bf16x2(pr[8 * c8], pr[8 * c8 + 1]), pack_bf16x2(pr[8 * c8 + 2], pr[8 * c8 + 3]),
+                                     pack_bf16x2(pr[8 * c8 + 4], pr[8 * c8 + 5]), pack_bf16x2(pr[8 * c8 + 6], pr[8 * c8 + 7]));
+          *reinterpret_cast<uint4*>(prow + sw128(row, h0 / 8 + c8)) = v;
+        }
+        if (H < SA_NP && hh == 1) {
+#pragma unroll
+          for (int c8 = H / 8; c8 < 8; ++c8) *reinterpret_cast<uint4*>(prow + sw128(row, c8)) = make_uint4(0u, 0u, 0u, 0u);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars.p_full[pb]);
@@ -310,51 +369,46 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
       }
       if (!ok) break;
       // ---- epilogue: head sums, normalise O^T, transpose through smem, store
-#pragma unroll
-      for (int h = 0; h < H; ++h) {
-        const float sm_h = warp_sum(lpart[h]);
-        if (lane == 0) sm->red[wq][h] = sm_h;
+      {
+        const float part = ReduceScatter<HT, 16>::run(lpart, lane);
+        if ((lane & (32 / HT - 1)) == 0) sm->red[q4][h0 + rs_index<HT>(lane)] = part;
       }
-      named_bar(2, 128);
-      if (s_lane < H) {
-        const float l = sm->red[0][s_lane] + sm->red[1][s_lane] + sm->red[2][s_lane] + sm->red[3][s_lane];
-        sm->inv_l[s_lane] = l > 0.f ? 1.f / l : 0.f;
-        if (lse != nullptr)
-          lse[g * H + s_lane] = l > 0.f ? (sm->mref[s_lane] + log2f(l)) * kLn2 : -INFINITY;
+      named_bar(2, SA_NSOFT);
+      if (tid < H) {
+        const float l = sm->red[0][tid] + sm->red[1][tid] + sm->red[2][tid] + sm->red[3][tid];
+        sm->inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
+        if (lse != nullptr) lse[g * H + tid] = l > 0.f ? (sm->mref[tid] + log2f(l)) * kLn2 : -INFINITY;
       }
-      bool wo = true;
-      if (s_lane == 0) wo = mbar_wait(&bars.o_full[ob], (uint32_t)((tk >> 1) & 1), abortp, errp, ERR_O_FULL);
-      ok = !named_bar_or(2, 128, !wo);
+      {
+        bool w = true;
+        if (tid == 0) w = mbar_wait(&bars.o_full[ob], (uint32_t)((tk >> 1) & 1), abortp, errp, ERR_O_FULL);
+        ok = !named_bar_or(2, SA_NSOFT, !w);
+      }
       if (!ok) break;
       tc_fence_after();
       uint16_t* stage_out = reinterpret_cast<uint16_t*>(q_s + qb * SA_Q_BYTES);   // [H][128] bf16
-      {
+      if (hh * 32 < H) {
         uint32_t r[32];
+        if (nt > 0) {
+          tmem_ld32(tmem + lane_off + 128 + ob * 64 + hh * 32, r);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int c0 = 0; c0 < H; c0 += 32) {
-          if (nt > 0) {
-            tmem_ld32(tmem + lane_off + 128 + ob * 64 + c0, r);
-            tmem_wait_ld();
-          } else {
+          for (int k = 0; k < 32; ++k) r[k] = 0u;
+        }
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = 0u;
-          }
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (c0 + k < H) {
-              const float v = __uint_as_float(r[k]) * sm->inv_l[c0 + k];
-              stage_out[(c0 + k) * kD + s_lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-            }
-          }
+        for (int k = 0; k < 32; ++k) {
+          const int h = hh * 32 + k;
+          if (h < H) stage_out[h * kD + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[k]) * sm->inv_l[h]));
         }
       }
       tc_fence_before();
       mbar_arrive(&bars.o_free[ob]);
-      named_bar(2, 128);
+      named_bar(2, SA_NSOFT);
       uint4* dst = reinterpret_cast<uint4*>(out + g * (long long)H * kD);
       const uint4* src = reinterpret_cast<const uint4*>(stage_out);
-      for (int x = s_lane; x < H * 16; x += 128) dst[x] = src[x];
-      named_bar(2, 128);
+      for (int x = tid; x < H * 16; x += SA_NSOFT) dst[x] = src[x];
+      named_bar(2, SA_NSOFT);
       mbar_arrive(&bars.q_empty[qb]);
     }
   } else {
@@ -362,7 +416,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
     if (lane == 0) {
       constexpr uint32_t ID_S = idesc_bf16(128, H, false, false);
       constexpr uint32_t ID_O = idesc_bf16(128, SA_NP, true, true);
-      int kv_it = 0, s_it = 0, p_it = 0;
+      int kv_it = 0, p_it = 0;
       bool ok = true;
       long long tk = 0;
       auto issue_pv = [&](int stage_prev, int j_prev, int ob) -> bool {
@@ -382,22 +436,23 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         ++p_it;
         return true;
       };
+      // S^T[j+2] reuses S buffer j & 1; it is issued after PV(j), which waits
+      // for p_full(j), so the softmax has finished reading S^T[j] by then.
+      int s_cnt = 0;
       for (long long g = blockIdx.x; g < n_tok && ok; g += gridDim.x, ++tk) {
         const int qb = (int)(tk & 1), ob = qb;
         if (!mbar_wait(&bars.tok_full[qb], (uint32_t)((tk >> 1) & 1), abortp, errp, ERR_TOK_FULL)) { ok = false; break; }
         const int nt = sm->n_tiles[qb];
-        if (tk >= 2 && nt > 0) {
-          // (waited only when this token writes O^T[ob])
-        }
-        if (tk >= 2) {
-          if (!mbar_wait(&bars.o_free[ob], (uint32_t)(((tk >> 1) - 1) & 1), abortp, errp, ERR_O_FREE)) { ok = false; break; }
+        if (tk >= 2 && !mbar_wait(&bars.o_free[ob], (uint32_t)(((tk >> 1) - 1) & 1), abortp, errp, ERR_O_FREE)) {
+          ok = false;
+          break;
         }
         const uint32_t q0 = smem_u32(q_s + qb * SA_Q_BYTES);
         int stage_prev = 0;
         for (int j = 0; j < nt; ++j) {
-          const int stage = kv_it % SA_STAGES, sb = s_it & 1;
+          const int stage = kv_it % SA_STAGES, sb = s_cnt & 1;
           if (!mbar_wait(&bars.kv_full[stage], (uint32_t)((kv_it / SA_STAGES) & 1), abortp, errp, ERR_KV_FULL)) { ok = false; break; }
-          if (s_it >= 2 && !mbar_wait(&bars.s_free[sb], (uint32_t)(((s_it >> 1) - 1) & 1), abortp, errp, ERR_S_FREE)) { ok = false; break; }
+          fence_proxy_async_smem();   // cp.async (generic proxy) writes -> tensor-core reads
           tc_fence_after();
           const uint32_t e0 = smem_u32(e_s + stage * SA_E_BYTES);
 #pragma unroll
@@ -407,7 +462,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
             mma_bf16(tmem + sb * 64, ad, bd, ID_S, k > 0 ? 1u : 0u);
           }
           mma_commit(&bars.s_full[sb]);
-          ++s_it;
+          ++s_cnt;
           if (j > 0 && !issue_pv(stage_prev, j - 1, ob)) { ok = false; break; }
           stage_prev = stage;
           ++kv_it;
@@ -424,7 +479,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 7) {
+  if (warp == SA_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
@@ -456,10 +511,13 @@ cslc_status launch_sparse_attn_sm100(const uint16_t* q, const uint16_t* kv, cons
   const long long n_tok = (long long)B * L;
   const int grid = (int)(n_tok < n_sm ? n_tok : n_sm);
   const float sl2 = scale * kLog2e;
+  CUtensorMap tm_q;   // q viewed as [B*L*H rows, 128] with a box of H rows x 64 dims
+  if (!sm100::make_tmap_bf16_2d(&tm_q, q, (uint64_t)n_tok * H, kD, kD * 2, (uint32_t)H, 64))
+    return set_error(CSLC_ERR_CUDA, "csa_sparse_attn: tensor map encoding failed");
   switch (H) {
-    case 16: sparse_attn_sm100_kernel<16><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse); break;
-    case 32: sparse_attn_sm100_kernel<32><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse); break;
-    default: sparse_attn_sm100_kernel<64><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse); break;
+    case 16: sparse_attn_sm100_kernel<16><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, tm_q); break;
+    case 32: sparse_attn_sm100_kernel<32><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, tm_q); break;
+    default: sparse_attn_sm100_kernel<64><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, tm_q); break;
   }
   return check_launch("sparse_attn_sm100_kernel");
 }

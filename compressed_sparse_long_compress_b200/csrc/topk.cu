@@ -139,33 +139,194 @@ __device__ void emit_selection(const uint32_t* keys, int n, const RadixResult& r
   }
 }
 
+constexpr int TK_BINS = 4096;   // value-range histogram bins (shares storage with the radix histogram)
+constexpr int TK_CAND = 2048;   // threshold-bin candidates handled in shared memory
+
+// Compacts the indices i in [0, n) with pred(i) into out[] in ascending order
+// (at most k are written): per-warp counts over contiguous segments, then a
+// second pass writes. wsum: TOPK_WARPS ints.
+template <class Pred>
+__device__ void emit_where(Pred pred, int n, int32_t* out, int k, int* wsum) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seg = ((n + TOPK_WARPS - 1) / TOPK_WARPS + 31) & ~31;
+  const int lo = warp * seg, hi = min(n, lo + seg);
+  const unsigned lt = (1u << lane) - 1u;
+  int cnt = 0;
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, i < hi && pred(i)));
+  }
+  if (lane == 0) wsum[warp] = cnt;
+  __syncthreads();
+  int run = 0;
+  for (int w = 0; w < warp; ++w) run += wsum[w];
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const bool sel = i < hi && pred(i);
+    const unsigned m = __ballot_sync(0xffffffffu, sel);
+    const int pos = run + __popc(m & lt);
+    if (sel && pos < k) out[pos] = i;
+    run += __popc(m);
+  }
+}
+
+__device__ __forceinline__ uint64_t composite(float v, int i) {
+  return ((uint64_t)float_key(v) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+}
+
+// One CTA per query row. Fast path: the row's min / max define 4096 equal
+// value bins; the bin holding the k-th largest score is found from a
+// histogram, every score in a higher bin is selected, and the remaining
+// slots go to the candidates of that bin ranked by (score desc, index asc).
+// Rows where that bin is too crowded (or the range is degenerate) take the
+// exact 8-bit radix select over order-preserving keys.
 __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
     const float* __restrict__ scores, int rows_in_buf, int row_begin, int L, int Nc, int m,
     int q_pos0, int topk, int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) uint32_t keys[];
-  __shared__ uint32_t hist[TOPK_WARPS * 256];
+  extern __shared__ __align__(16) float vals[];
+  __shared__ uint32_t hist[TK_BINS];
+  __shared__ uint64_t cand[TK_CAND];
+  __shared__ float red[2][TOPK_WARPS];
+  __shared__ uint32_t wtot[TOPK_WARPS];
   __shared__ int bcast[4];
   __shared__ int wsum[2 * TOPK_WARPS];
+  __shared__ int n_cand;
+  __shared__ uint64_t thr_comp;
   const int r = row_begin + blockIdx.x;
   const int b = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nv = n_visible((long long)q_pos0 + r, m, Nc);
   int32_t* out = idx + ((size_t)b * L + r) * topk;
   if (nv <= topk) {
     for (int j = tid; j < topk; j += TOPK_THREADS) out[j] = j < nv ? j : -1;
     return;
   }
+  for (int x = tid; x < TK_BINS; x += TOPK_THREADS) hist[x] = 0;
+  if (tid == 0) n_cand = 0;
+  // load the visible scores, tracking min / max
   const float* srow = scores + ((size_t)b * rows_in_buf + (r - row_begin)) * (size_t)Nc;
+  float vmin = INFINITY, vmax = -INFINITY;
+  int done = 0;
   if ((Nc & 3) == 0) {
     const int n4 = nv >> 2;
     for (int j = tid; j < n4; j += TOPK_THREADS) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(srow) + j);
-      reinterpret_cast<uint4*>(keys)[j] = make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w));
+      reinterpret_cast<float4*>(vals)[j] = v;
+      vmin = fminf(fminf(vmin, v.x), fminf(fminf(v.y, v.z), v.w));
+      vmax = fmaxf(fmaxf(vmax, v.x), fmaxf(fmaxf(v.y, v.z), v.w));
     }
-    for (int j = (n4 << 2) + tid; j < nv; j += TOPK_THREADS) keys[j] = float_key(__ldcs(srow + j));
-  } else {
-    for (int j = tid; j < nv; j += TOPK_THREADS) keys[j] = float_key(__ldcs(srow + j));
+    done = n4 << 2;
   }
+  for (int j = done + tid; j < nv; j += TOPK_THREADS) {
+    const float v = __ldcs(srow + j);
+    vals[j] = v;
+    vmin = fminf(vmin, v);
+    vmax = fmaxf(vmax, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  }
+  if (lane == 0) { red[0][warp] = vmin; red[1][warp] = vmax; }
+  __syncthreads();
+  float lo = red[0][0], hi = red[1][0];
+  for (int w = 1; w < TOPK_WARPS; ++w) { lo = fminf(lo, red[0][w]); hi = fmaxf(hi, red[1][w]); }
+  const float span = hi - lo;
+  bool fast = span > 0.f && isfinite(span);
+  const float bscale = fast ? ((float)TK_BINS - 0.5f) / span : 0.f;
+  auto bin_of = [&](float v) { return min(TK_BINS - 1, (int)((v - lo) * bscale)); };
+  int T = 0, remaining = 0;
+  if (fast) {
+    for (int j = tid; j < nv; j += TOPK_THREADS) atomicAdd(&hist[bin_of(vals[j])], 1u);
+    __syncthreads();
+    // thread t owns bins 4095 - 8t .. 4088 - 8t (descending); find the bin holding the k-th largest
+    uint32_t c[8], s = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { c[j] = hist[TK_BINS - 1 - 8 * tid - j]; s += c[j]; }
+    uint32_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += wtot[w];
+    incl += before;
+    const uint32_t excl = incl - s;
+    if (excl < (uint32_t)topk && incl >= (uint32_t)topk) {
+      uint32_t above = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (above + c[j] >= (uint32_t)topk) {
+          bcast[0] = TK_BINS - 1 - 8 * tid - j;
+          bcast[1] = (int)above;
+          bcast[2] = (int)c[j];
+          break;
+        }
+        above += c[j];
+      }
+    }
+    __syncthreads();
+    T = bcast[0];
+    remaining = topk - bcast[1];
+    const int cntT = bcast[2];
+    if (cntT == remaining) {
+      emit_where([&](int i) { return bin_of(vals[i]) >= T; }, nv, out, topk, wsum);
+      return;
+    }
+    if (cntT > TK_CAND) fast = false;
+  }
+  if (fast) {
+    // candidates of bin T, then the remaining-th largest (score desc, index asc)
+    for (int j = tid; j < nv; j += TOPK_THREADS) {
+      const float v = vals[j];
+      if (bin_of(v) == T) cand[atomicAdd(&n_cand, 1)] = composite(v, j);
+    }
+    __syncthreads();
+    const int C = n_cand;
+    if (C <= TOPK_THREADS) {
+      if (tid < C) {
+        const uint64_t me = cand[tid];
+        int rank = 0;
+        for (int j = 0; j < C; ++j) rank += cand[j] > me;
+        if (rank == remaining - 1) thr_comp = me;
+      }
+    } else {
+      int P = 1;
+      while (P < C) P <<= 1;
+      for (int j = C + tid; j < P; j += TOPK_THREADS) cand[j] = 0ull;
+      __syncthreads();
+      for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          for (int i = tid; i < P; i += TOPK_THREADS) {
+            const int jx = i ^ stride;
+            if (jx > i) {
+              const bool desc = (i & size) == 0;
+              const uint64_t a = cand[i], c2 = cand[jx];
+              if ((a < c2) == desc) { cand[i] = c2; cand[jx] = a; }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      if (tid == 0) thr_comp = cand[remaining - 1];
+    }
+    __syncthreads();
+    const uint64_t tc = thr_comp;
+    emit_where([&](int i) {
+      const float v = vals[i];
+      const int bi = bin_of(v);
+      return bi > T || (bi == T && composite(v, i) >= tc);
+    }, nv, out, topk, wsum);
+    return;
+  }
+  // exact radix select over order-preserving keys (degenerate value ranges)
+  __syncthreads();
+  uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
+  for (int j = tid; j < nv; j += TOPK_THREADS) keys[j] = float_key(vals[j]);
   __syncthreads();
   const RadixResult rr = radix_select(keys, nv, topk, hist, bcast);
   emit_selection(keys, nv, rr, out, topk, wsum);
@@ -181,7 +342,7 @@ cslc_status launch_topk_rows(const float* scores, int rows_in_buf, int row_begin
   cudaGetDevice(&dev);
   if (configured_for != dev) {
     cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
+                         192 * 1024);
     configured_for = dev;
   }
   dim3 grid(row_end - row_begin, B);
