@@ -38,6 +38,7 @@ cslc_status launch_dense_attn(const uint16_t*, const uint16_t*, int, int, int, i
                               uint16_t*, float*, cudaStream_t);
 size_t decode_workspace_bytes(const cslc_decode_layer*, int, int, int);
 int sparse_attn_sm100_read_error();
+int dense_attn_sm100_read_error();
 size_t decode_topk_workspace_bytes(int, int, int);
 cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*, size_t, cudaStream_t);
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
@@ -85,6 +86,9 @@ cslc_status cslc_sync_status(cslc_stream_t stream) {
   const int code = sparse_attn_sm100_read_error();
   if (code != 0)
     return set_error(CSLC_ERR_DEVICE_CHECK, "csa_sparse_attn: a pipeline wait timed out (code %d)", code);
+  const int code2 = dense_attn_sm100_read_error();
+  if (code2 != 0)
+    return set_error(CSLC_ERR_DEVICE_CHECK, "hca_dense_attn: a pipeline wait timed out (code %d)", code2);
   return CSLC_OK;
 }
 

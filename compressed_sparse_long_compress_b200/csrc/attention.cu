@@ -265,10 +265,17 @@ cslc_status launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const int3
   return check_launch("attention_kernel<sparse>");
 }
 
+bool dense_attn_sm100_supported(int H);
+cslc_status launch_dense_attn_sm100(const uint16_t*, const uint16_t*, int, int, int, int, int, int, float,
+                                    uint16_t*, float*, cudaStream_t);
+
 cslc_status launch_dense_attn(const uint16_t* q, const uint16_t* kv, int B, int L, int H, int Nc,
                               int m, int q_pos0, float scale, uint16_t* out, float* lse,
                               cudaStream_t stream) {
   if (B == 0 || L == 0) return CSLC_OK;
+  // tcgen05 kernel when 128 rows hold whole tokens (H divides 128); other head counts below
+  if (dense_attn_sm100_supported(H))
+    return launch_dense_attn_sm100(q, kv, B, L, H, Nc, m, q_pos0, scale, out, lse, stream);
   if (H <= 64) {
     attn_configure<false, 2>();
     // 2 tokens per CTA when H <= 64 (<= 8 warps)
