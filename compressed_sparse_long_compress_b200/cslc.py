@@ -27,7 +27,7 @@ ABI_SYMBOLS = [
     "cslc_abi_version", "cslc_last_error", "cslc_sync_status", "csa_compress", "hca_compress",
     "csa_indexer_topk_workspace_bytes", "csa_indexer_topk", "csa_topk", "csa_sparse_attn",
     "hca_dense_attn", "cslc_quantize_kv_mixed", "cslc_decode_workspace_bytes", "cslc_decode_step",
-    "cslc_decode_topk_workspace_bytes", "cslc_decode_topk",
+    "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc",
 ]
 
 
@@ -70,6 +70,7 @@ def _load():
                                      P, c_size_t, P]),
         "cslc_decode_topk_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
         "cslc_decode_topk": (c_int, [P, P, c_int, c_int, c_int, P, P, c_size_t, P]),
+        "cslc_decode_topk_noalloc": (c_int, [P, P, c_int, c_int, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -301,4 +302,16 @@ def decode_topk(scores, n_entries, topk: int, idx=None, stream=None):
     ws = torch.empty(max(nbytes, 16), dtype=U8, device=scores.device)
     _check(LIB.cslc_decode_topk(_ptr(scores), _ptr(n_entries), B, n_max, topk, _ptr(idx), _ptr(ws),
                                 ws.numel(), _stream(stream)))
+    return idx
+
+
+def decode_topk_noalloc(scores, n_entries, topk: int, idx=None, stream=None):
+    """decode_topk using the library's static scratch instead of a workspace
+    (for callers that cannot allocate device memory; see include/cslc.h)."""
+    B, n_max = scores.shape
+    _need(scores, F32, "scores"); _need(n_entries, I32, "n_entries", (B,))
+    if idx is None:
+        idx = torch.empty(B, topk, dtype=I32, device=scores.device)
+    _need(idx, I32, "idx", (B, topk))
+    _check(LIB.cslc_decode_topk_noalloc(_ptr(scores), _ptr(n_entries), B, n_max, topk, _ptr(idx), _stream(stream)))
     return idx

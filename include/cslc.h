@@ -219,6 +219,29 @@ cslc_status cslc_decode_topk(const float* scores, const int32_t* n_entries, int 
                              int topk, int32_t* idx, void* ws, size_t ws_bytes,
                              cslc_stream_t stream);
 
+/* ------------------------------------------------------------------------ */
+/* The decode top-k without a caller workspace (the source pages have no
+ * counterpart: this is a deployment convenience of the library).
+ *
+ * For callers that cannot call cudaMalloc -- e.g. a serving process whose
+ * device memory is fully planned at start-up, code where an allocation would
+ * synchronise the device, or a C caller with no device allocator. Same
+ * arguments, selection rule and result as cslc_decode_topk, but the scratch
+ * comes from one static device array of 16 MiB inside the library, held by
+ * every GPU that loads the library until the process exits. The call
+ * allocates nothing.
+ *   - Requires cslc_decode_topk_workspace_bytes(B, n_max, topk) <= 16 MiB
+ *     (e.g. B = 8 with n_max up to ~245,000); larger calls return
+ *     CSLC_ERR_WORKSPACE without launching anything.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the array and it keeps the last call's contents (the
+ *     parts that must start at zero are cleared on the stream by each call);
+ *     calls whose work overlaps on the GPU (e.g. on two streams at once) race.
+ */
+cslc_status cslc_decode_topk_noalloc(const float* scores, const int32_t* n_entries, int B, int n_max,
+                                     int topk, int32_t* idx, cslc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
