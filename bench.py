@@ -55,7 +55,7 @@ def load_peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples (every 200 ms) during the timed region."""
+    """nvidia-smi clock / throttle samples (every 50 ms) during the timed region."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -72,7 +72,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
         return self
@@ -189,9 +189,10 @@ class CsaPrefill:
 
     def roofline(self, kernel_ms, peaks):
         ach = self.flops_attn / (kernel_ms * 1e-3) / 1e12
-        return {"kernel": "csa_sparse_attn (attention_kernel<sparse>)", "bound": "tensor",
+        return {"kernel": "csa_sparse_attn (sparse_attn_sm100_kernel<64>)", "bound": "tensor",
                 "achieved": round(ach, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": None,
+                "frac": round(ach / peaks["bf16_tflops"], 4),
+                "traffic": measured_traffic("sparse", self.units),
                 "algorithmic_flops_per_launch": self.flops_attn, "peak_source": peaks["source"] + " (burst)"}
 
     def config(self):
@@ -234,9 +235,9 @@ class HcaPrefill:
 
     def roofline(self, kernel_ms, peaks):
         ach = self.flops_attn / (kernel_ms * 1e-3) / 1e12
-        return {"kernel": "hca_dense_attn (attention_kernel<dense>)", "bound": "tensor", "achieved": round(ach, 2),
+        return {"kernel": "hca_dense_attn (dense_attn_sm100_kernel)", "bound": "tensor", "achieved": round(ach, 2),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
-                "traffic": None, "algorithmic_flops_per_launch": self.flops_attn,
+                "traffic": measured_traffic("dense", self.units), "algorithmic_flops_per_launch": self.flops_attn,
                 "peak_source": peaks["source"] + " (burst)"}
 
     def config(self):
@@ -383,6 +384,68 @@ def measure(name, C, args, world, rank, local, peaks, flush, with_e2e=True):
     return res
 
 
+# ------------------------------------------------------------ ncu cases
+
+def profile_case(name):
+    """One small case of a kernel for an ncu capture (inputs larger than L2,
+    a few GB on the device): builds seeded inputs and calls the entry twice."""
+    from compressed_sparse_long_compress_b200 import cslc as C
+    dev = torch.device("cuda", 0)
+    if name == "sparse_attn_L8192":
+        L, H, n_c, k = 8192, 64, 16384, 1024
+        q = W.randn_bf16((1, L, H, 128), 1, device=dev)
+        e = W.randn_bf16((1, n_c, 128), 2, device=dev, std=0.4)
+        g = torch.Generator(device=dev)
+        g.manual_seed(3)
+        idx = torch.sort(torch.rand(1, L, n_c, device=dev, generator=g).topk(k, dim=-1).indices.int(),
+                         dim=-1).values.contiguous()
+        out = torch.empty_like(q)
+        for _ in range(2):
+            C.csa_sparse_attn(q, e, idx, 1 / math.sqrt(128), out=out)
+    elif name == "dense_attn_L65536":
+        L, H = 65536, 64
+        q = W.randn_bf16((1, L, H, 128), 1, device=dev)
+        e = W.randn_bf16((1, L // 128, 128), 2, device=dev, std=0.4)
+        out = torch.empty_like(q)
+        for _ in range(2):
+            C.hca_dense_attn(q, e, m_prime=128, scale=1 / math.sqrt(128), out=out)
+    elif name == "topk_L8192":
+        L, n_c, k = 8192, 16384, 1024
+        scores = W.rand_f32((1, L, n_c), seed=4, device=dev)
+        idx = torch.empty(1, L, k, dtype=torch.int32, device=dev)
+        for _ in range(2):
+            C.csa_topk(scores, m=4, topk=k, q_pos0=4 * n_c, idx=idx)   # every row sees all entries
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    C.sync_status()
+    print("ok", name)
+
+
+# DRAM bytes (read + write) per launch from one ncu capture of a smaller case
+# (profiles/), scaled by the tokens a launch processes; valid only while the
+# kernel source is the one that was measured.
+MEASURED_TRAFFIC = {
+    "sparse": {"src": "sparse_attn_sm100.cu",
+               "sha256": "7ed05fe7c53211ef9cd7a027600107ce2aa0bc39fe9c860f85035ba4bc5adc08",
+               "bytes_per_token": (172.030464e6 + 101.147136e6) / 8192},
+    "dense": {"src": "dense_attn_sm100.cu",
+              "sha256": "dd8fec45b42bbc05b73ad2872a7b3c0f8d46e1ba28a96c6b8f4416c7f0dcf2ce",
+              "bytes_per_token": (1.074034e9 + 1.024294e9) / 65536},
+}
+
+
+def measured_traffic(kind, tokens):
+    import hashlib
+    t = MEASURED_TRAFFIC[kind]
+    path = os.path.join(ROOT, "compressed_sparse_long_compress_b200", "csrc", t["src"])
+    try:
+        h = hashlib.sha256(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return t["bytes_per_token"] * tokens if h == t["sha256"] else None
+
+
 # ----------------------------------------------------------- CPU baseline
 
 def blas_threads():
@@ -490,13 +553,18 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="csa_prefill", choices=list(W.WORKLOADS))
     ap.add_argument("--secondary", default="all", choices=["none", "all"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192"],
+                    help="run one small kernel case for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         args.warmup = 3
 

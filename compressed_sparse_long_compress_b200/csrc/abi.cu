@@ -44,7 +44,7 @@ cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*,
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
 
 constexpr int kMaxTopk = 2048;
-constexpr int kMaxPrefillTopkNc = 49152;   // a row of scores must fit in shared memory
+constexpr int kMaxPrefillTopkNc = 45056;   // a row of scores must fit in shared memory
 
 static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 

@@ -78,9 +78,9 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
   if (tid == 0) {
     mbar_init(&bars.q_full, 1); mbar_init(&bars.q_empty, 1);
     for (int s = 0; s < DA_STAGES; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&bars.s_full[i], 1); mbar_init(&bars.p_full[i], 128); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&bars.s_full[i], 1); mbar_init(&bars.p_full[i], 4); }
     mbar_init(&bars.pv_done, 1);
-    mbar_init(&bars.o_full, 1); mbar_init(&bars.o_free, 128);
+    mbar_init(&bars.o_full, 1); mbar_init(&bars.o_free, 4);
     mbar_init(&bars.final_bar, 1);
     sm->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -289,7 +289,8 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
         lrow += psum;
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars.p_full[pb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[pb]);
         ++s_it;
         ++p_it;
       }
@@ -326,7 +327,8 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
       }
       if (row_ok && lse != nullptr) lse[orow] = lrow > 0.f ? (mrow + log2f(lrow)) * kLn2 : -INFINITY;
       tc_fence_before();
-      mbar_arrive(&bars.o_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.o_free);
     }
   }
   tc_fence_before();

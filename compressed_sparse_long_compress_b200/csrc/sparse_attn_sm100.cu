@@ -82,7 +82,7 @@ struct SaSmall {
   __align__(16) float mref[SA_NP];   // running max per head (log2 units of c*S)
   __align__(16) float alpha[SA_NP];
   __align__(16) float inv_l[SA_NP];
-  float red[4][SA_NP];               // per lane-quadrant partials
+  __align__(16) float red[4][SA_NP];  // per lane-quadrant partials
 };
 
 // Reduce-scatter of N per-lane values over the warp: returns, in every lane,
@@ -147,10 +147,10 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
   if (tid == 0) {
     for (int s = 0; s < SA_STAGES; ++s) { mbar_init(&bars.kv_full[s], SA_NPROD); mbar_init(&bars.kv_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.tok_full[i], 1); mbar_init(&bars.q_empty[i], SA_NSOFT);
+      mbar_init(&bars.tok_full[i], 1); mbar_init(&bars.q_empty[i], SA_NSOFT / 32);
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.p_full[i], SA_NSOFT);
-      mbar_init(&bars.o_full[i], 1); mbar_init(&bars.o_free[i], SA_NSOFT);
+      mbar_init(&bars.p_full[i], SA_NSOFT / 32);
+      mbar_init(&bars.o_full[i], 1); mbar_init(&bars.o_free[i], SA_NSOFT / 32);
     }
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.final_bar, 1);
@@ -259,47 +259,52 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
 #pragma unroll
       for (int h = 0; h < HT; ++h) lpart[h] = 0.f;
 
+      float negm[HT];                        // -m[h] (log2 units) of this thread's heads
+#pragma unroll
+      for (int h = 0; h < HT; ++h) negm[h] = INFINITY;
       for (int j = 0; j < nt; ++j) {
         const int sb = s_it & 1, pb = p_it & 1;
-        {
-          bool w = true;
-          if (tid == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
-          ok = !named_bar_or(2, SA_NSOFT, !w);
-        }
-        if (!ok) break;
-        tc_fence_after();
-        float raw[HT];
-        {
+        // each warp waits for S on its own; a timeout anywhere raises the abort
+        // flag, which every thread reads after the tile's CTA-wide barrier
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
+        w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+        const int slot = j * SA_TILE + row;
+        const bool valid = slot < topk && is[slot] >= 0;
+        float v[HT];
+        float pmax = 0.f;
+        if (w) {
+          tc_fence_after();
           uint32_t r[32];
           tmem_ld32(tmem + lane_off + sb * 64 + h0, r);
           tmem_wait_ld();
+          if (valid && j > 0) {
 #pragma unroll
-          for (int h = 0; h < HT; ++h) raw[h] = __uint_as_float(r[h]);
-        }
-        const int slot = j * SA_TILE + row;
-        const bool valid = slot < topk && is[slot] >= 0;
-        float pr[HT];
-        bool slow = (j == 0);
-        if (!slow) {
-          float pmax = 0.f;
-#pragma unroll
-          for (int h4 = 0; h4 < HT; h4 += 4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(&sm->mref[h0 + h4]);
-            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              pr[h4 + k] = valid ? ex2_approx(fmaf(raw[h4 + k], scale_log2, -mm[k])) : 0.f;
-              pmax = fmaxf(pmax, pr[h4 + k]);
+            for (int h = 0; h < HT; ++h) {
+              v[h] = ex2_approx(fmaf(__uint_as_float(r[h]), scale_log2, negm[h]));
+              pmax = fmaxf(pmax, v[h]);
             }
-          }
-          slow = named_bar_or(3, SA_NSOFT, pmax > SA_OVERFLOW);
-        }
-        if (slow) {
-          // exact per-head maximum of this tile (raw scores; scaled below)
+          } else {
 #pragma unroll
-          for (int h = 0; h < HT; ++h) {
-            const float mx = warp_redux_max(valid ? raw[h] : -INFINITY);
-            if (lane == 0) sm->red[q4][h0 + h] = mx;
+            for (int h = 0; h < HT; ++h) v[h] = 0.f;
+          }
+        }
+        // j == 0 always takes the exact-max path (negm starts at +inf)
+        const bool slow = named_bar_or(3, SA_NSOFT, j == 0 || !(pmax <= SA_OVERFLOW) || !w);
+        if (*abortp) { ok = false; break; }
+        if (slow) {
+          // exact per-head maximum of this tile from S (still intact: the next
+          // S into this buffer waits for this tile's p_full)
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + sb * 64 + h0, r);
+          tmem_wait_ld();
+          float mx[HT];
+#pragma unroll
+          for (int h = 0; h < HT; ++h) mx[h] = warp_redux_max(valid ? __uint_as_float(r[h]) : -INFINITY);
+          if (lane == 0) {
+#pragma unroll
+            for (int h4 = 0; h4 < HT; h4 += 4)
+              *reinterpret_cast<float4*>(&sm->red[q4][h0 + h4]) = make_float4(mx[h4], mx[h4 + 1], mx[h4 + 2], mx[h4 + 3]);
           }
           if (tid == 0) sm->any_rescale = 0;
           named_bar(2, SA_NSOFT);
@@ -318,44 +323,44 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
           }
           named_bar(2, SA_NSOFT);
 #pragma unroll
-          for (int h = 0; h < HT; ++h) lpart[h] *= sm->alpha[h0 + h];
+          for (int h4 = 0; h4 < HT; h4 += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(&sm->mref[h0 + h4]);
+            const float4 a4 = *reinterpret_cast<const float4*>(&sm->alpha[h0 + h4]);
+            negm[h4] = m4.x == -INFINITY ? INFINITY : -m4.x;
+            negm[h4 + 1] = m4.y == -INFINITY ? INFINITY : -m4.y;
+            negm[h4 + 2] = m4.z == -INFINITY ? INFINITY : -m4.z;
+            negm[h4 + 3] = m4.w == -INFINITY ? INFINITY : -m4.w;
+            lpart[h4] *= a4.x; lpart[h4 + 1] *= a4.y; lpart[h4 + 2] *= a4.z; lpart[h4 + 3] *= a4.w;
+          }
           if (sm->any_rescale) {
             // O^T must be stable: the previous tile's PV has to be complete
-            {
-              bool w = true;
-              if (tid == 0) w = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
-              ok = !named_bar_or(2, SA_NSOFT, !w);
-            }
+            bool w2 = true;
+            if (tid == 0) w2 = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
+            ok = !named_bar_or(2, SA_NSOFT, !w2);
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[32];
+            uint32_t o[32];
             const uint32_t oc = tmem + lane_off + 128 + ob * 64 + hh * 32;
-            tmem_ld32(oc, r);
+            tmem_ld32(oc, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * sm->alpha[hh * 32 + k]);
-            tmem_st32(oc, r);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * sm->alpha[hh * 32 + k]);
+            tmem_st32(oc, o);
             tmem_wait_st();
           }
 #pragma unroll
-          for (int h4 = 0; h4 < HT; h4 += 4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(&sm->mref[h0 + h4]);
-            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              pr[h4 + k] = valid ? ex2_approx(fmaf(raw[h4 + k], scale_log2, -mm[k])) : 0.f;
-          }
+          for (int h = 0; h < HT; ++h) v[h] = valid ? ex2_approx(fmaf(__uint_as_float(r[h]), scale_log2, negm[h])) : 0.f;
         }
 #pragma unroll
-        for (int h = 0; h < HT; ++h) lpart[h] += pr[h];
+        for (int h = 0; h < HT; ++h) lpart[h] += v[h];
         // P^T row: this thread's heads h0 .. h0+HT-1 (chunks of 8 heads); the
         // second head half also zero-fills the padding heads H .. 63
         uint8_t* prow = p_s + pb * SA_P_BYTES;
 #pragma unroll
         for (int c8 = 0; c8 < HT / 8; ++c8) {
-          const uint4 v = make_uint4(pack_bf16x2(pr[8 * c8], pr[8 * c8 + 1]), pack_bf16x2(pr[8 * c8 + 2], pr[8 * c8 + 3]),
-                                     pack_bf16x2(pr[8 * c8 + 4], pr[8 * c8 + 5]), pack_bf16x2(pr[8 * c8 + 6], pr[8 * c8 + 7]));
-          *reinterpret_cast<uint4*>(prow + sw128(row, h0 / 8 + c8)) = v;
+          const uint4 pv = make_uint4(pack_bf16x2(v[8 * c8], v[8 * c8 + 1]), pack_bf16x2(v[8 * c8 + 2], v[8 * c8 + 3]),
+                                      pack_bf16x2(v[8 * c8 + 4], v[8 * c8 + 5]), pack_bf16x2(v[8 * c8 + 6], v[8 * c8 + 7]));
+          *reinterpret_cast<uint4*>(prow + sw128(row, h0 / 8 + c8)) = pv;
         }
         if (H < SA_NP && hh == 1) {
 #pragma unroll
@@ -363,7 +368,8 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars.p_full[pb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[pb]);
         ++s_it;
         ++p_it;
       }
@@ -403,13 +409,14 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars.o_free[ob]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.o_free[ob]);
       named_bar(2, SA_NSOFT);
       uint4* dst = reinterpret_cast<uint4*>(out + g * (long long)H * kD);
       const uint4* src = reinterpret_cast<const uint4*>(stage_out);
       for (int x = tid; x < H * 16; x += SA_NSOFT) dst[x] = src[x];
       named_bar(2, SA_NSOFT);
-      mbar_arrive(&bars.q_empty[qb]);
+      if (lane == 0) mbar_arrive(&bars.q_empty[qb]);
     }
   } else {
     // ------------------------------------------------------------ MMA issuer

@@ -142,50 +142,36 @@ __device__ void emit_selection(const uint32_t* keys, int n, const RadixResult& r
 constexpr int TK_BINS = 4096;   // value-range histogram bins (shares storage with the radix histogram)
 constexpr int TK_CAND = 2048;   // threshold-bin candidates handled in shared memory
 
-// Compacts the indices i in [0, n) with pred(i) into out[] in ascending order
-// (at most k are written): per-warp counts over contiguous segments, then a
-// second pass writes. wsum: TOPK_WARPS ints.
-template <class Pred>
-__device__ void emit_where(Pred pred, int n, int32_t* out, int k, int* wsum) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int seg = ((n + TOPK_WARPS - 1) / TOPK_WARPS + 31) & ~31;
-  const int lo = warp * seg, hi = min(n, lo + seg);
-  const unsigned lt = (1u << lane) - 1u;
-  int cnt = 0;
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    cnt += __popc(__ballot_sync(0xffffffffu, i < hi && pred(i)));
-  }
-  if (lane == 0) wsum[warp] = cnt;
-  __syncthreads();
-  int run = 0;
-  for (int w = 0; w < warp; ++w) run += wsum[w];
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    const bool sel = i < hi && pred(i);
-    const unsigned m = __ballot_sync(0xffffffffu, sel);
-    const int pos = run + __popc(m & lt);
-    if (sel && pos < k) out[pos] = i;
-    run += __popc(m);
-  }
-}
-
 __device__ __forceinline__ uint64_t composite(float v, int i) {
   return ((uint64_t)float_key(v) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
 }
 
-// One CTA per query row. Fast path: the row's min / max define 4096 equal
-// value bins; the bin holding the k-th largest score is found from a
-// histogram, every score in a higher bin is selected, and the remaining
-// slots go to the candidates of that bin ranked by (score desc, index asc).
-// Rows where that bin is too crowded (or the range is degenerate) take the
-// exact 8-bit radix select over order-preserving keys.
+// One CTA per query row.
+// Fast path (touches each score a few times with cheap work):
+//   1. each thread loads its scores with all loads in flight; one of them per
+//      thread, spread over the row, fixes a value range [lo, hi];
+//   2. one pass over those registers bins every score into 4096 equal
+//      bins of that range (scores outside clamp to the edge bins, which keeps
+//      the binning monotone), adds it to a shared histogram and keeps its
+//      16-bit bin in shared memory;
+//   3. the bin T holding the k-th largest score is found by a block scan; all
+//      scores in higher bins are selected; when bin T must be split, its
+//      scores are re-read and ranked exactly by (score desc, index asc) and the
+//      chosen ones are marked in a bitmap;
+//   4. two passes over the 16-bit bins (eight per 16-byte read) count the
+//      selection per warp segment and then write the indices in ascending order.
+// Rows whose sampled range is degenerate, or whose threshold bin is too
+// crowded, take the exact 8-bit radix select over order-preserving keys.
+constexpr int TK_MAXN = 45056;   // longest row (entries) the shared memory holds
+constexpr int TK_REG = 8;        // float4 loads per thread held in registers (power of two)
+
 __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
     const float* __restrict__ scores, int rows_in_buf, int row_begin, int L, int Nc, int m,
     int q_pos0, int topk, int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) float vals[];
+  extern __shared__ __align__(16) uint32_t dyn[];          // n words: bins (fast) or keys (fallback)
   __shared__ uint32_t hist[TK_BINS];
   __shared__ uint64_t cand[TK_CAND];
+  __shared__ uint32_t selbits[TK_MAXN / 32];
   __shared__ float red[2][TOPK_WARPS];
   __shared__ uint32_t wtot[TOPK_WARPS];
   __shared__ int bcast[4];
@@ -201,50 +187,79 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
     for (int j = tid; j < topk; j += TOPK_THREADS) out[j] = j < nv ? j : -1;
     return;
   }
-  for (int x = tid; x < TK_BINS; x += TOPK_THREADS) hist[x] = 0;
-  if (tid == 0) n_cand = 0;
-  // load the visible scores, tracking min / max
   const float* srow = scores + ((size_t)b * rows_in_buf + (r - row_begin)) * (size_t)Nc;
-  float vmin = INFINITY, vmax = -INFINITY;
-  int done = 0;
-  if ((Nc & 3) == 0) {
-    const int n4 = nv >> 2;
-    for (int j = tid; j < n4; j += TOPK_THREADS) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(srow) + j);
-      reinterpret_cast<float4*>(vals)[j] = v;
-      vmin = fminf(fminf(vmin, v.x), fminf(fminf(v.y, v.z), v.w));
-      vmax = fmaxf(fmaxf(vmax, v.x), fmaxf(fmaxf(v.y, v.z), v.w));
-    }
-    done = n4 << 2;
-  }
-  for (int j = done + tid; j < nv; j += TOPK_THREADS) {
-    const float v = __ldcs(srow + j);
-    vals[j] = v;
-    vmin = fminf(vmin, v);
-    vmax = fmaxf(vmax, v);
-  }
+  uint16_t* bins = reinterpret_cast<uint16_t*>(dyn);
+  for (int x = tid; x < TK_BINS; x += TOPK_THREADS) hist[x] = 0;
+  for (int x = tid; x < (nv + 31) / 32; x += TOPK_THREADS) selbits[x] = 0;
+  if (tid == 0) n_cand = 0;
+  // 1. the row's first TK_REG * 4 * TOPK_THREADS scores go to registers with all
+  //    loads in flight at once; one of them per thread (spread over the row)
+  //    samples the value range
+  const bool vec = (Nc & 3) == 0;
+  const int n4 = vec ? (nv >> 2) : 0;
+  float4 rv[TK_REG];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  for (int i = 0; i < TK_REG; ++i) {
+    const int j = tid + i * TOPK_THREADS;
+    rv[i] = j < n4 ? __ldcs(reinterpret_cast<const float4*>(srow) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (lane == 0) { red[0][warp] = vmin; red[1][warp] = vmax; }
+  {
+    const int si = tid & (TK_REG - 1);
+    const int sj = tid + si * TOPK_THREADS;
+    float v;
+    if (vec && sj < n4) {
+      v = rv[0].x;
+#pragma unroll
+      for (int i = 1; i < TK_REG; ++i) if (i == si) v = rv[i].x;
+    } else {
+      v = __ldg(srow + (int)(((long long)tid * nv) / TOPK_THREADS));
+    }
+    float vmin = v, vmax = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (lane == 0) { red[0][warp] = vmin; red[1][warp] = vmax; }
+  }
   __syncthreads();
   float lo = red[0][0], hi = red[1][0];
   for (int w = 1; w < TOPK_WARPS; ++w) { lo = fminf(lo, red[0][w]); hi = fmaxf(hi, red[1][w]); }
   const float span = hi - lo;
-  bool fast = span > 0.f && isfinite(span);
+  bool fast = span > 0.f && isfinite(span) && nv <= TK_MAXN;
   const float bscale = fast ? ((float)TK_BINS - 0.5f) / span : 0.f;
-  auto bin_of = [&](float v) { return min(TK_BINS - 1, (int)((v - lo) * bscale)); };
+  auto bin_of = [&](float v) { return min(TK_BINS - 1, max(0, (int)((v - lo) * bscale))); };
   int T = 0, remaining = 0;
+  bool take_all = false;
   if (fast) {
-    for (int j = tid; j < nv; j += TOPK_THREADS) atomicAdd(&hist[bin_of(vals[j])], 1u);
-    __syncthreads();
-    // thread t owns bins 4095 - 8t .. 4088 - 8t (descending); find the bin holding the k-th largest
-    uint32_t c[8], s = 0;
+    // 2. bin every score (registers / global -> histogram + 16-bit bins)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { c[j] = hist[TK_BINS - 1 - 8 * tid - j]; s += c[j]; }
-    uint32_t incl = s;
+    for (int i = 0; i < TK_REG; ++i) {
+      const int j = tid + i * TOPK_THREADS;
+      if (j < n4) {
+        const float4 v = rv[i];
+        const int b0 = bin_of(v.x), b1 = bin_of(v.y), b2 = bin_of(v.z), b3 = bin_of(v.w);
+        atomicAdd(&hist[b0], 1u); atomicAdd(&hist[b1], 1u); atomicAdd(&hist[b2], 1u); atomicAdd(&hist[b3], 1u);
+        reinterpret_cast<uint2*>(bins)[j] = make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+      }
+    }
+    for (int j = tid + TK_REG * TOPK_THREADS; j < n4; j += TOPK_THREADS) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(srow) + j);
+      const int b0 = bin_of(v.x), b1 = bin_of(v.y), b2 = bin_of(v.z), b3 = bin_of(v.w);
+      atomicAdd(&hist[b0], 1u); atomicAdd(&hist[b1], 1u); atomicAdd(&hist[b2], 1u); atomicAdd(&hist[b3], 1u);
+      reinterpret_cast<uint2*>(bins)[j] = make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+    }
+    for (int j = (n4 << 2) + tid; j < nv; j += TOPK_THREADS) {
+      const int bb = bin_of(__ldcs(srow + j));
+      atomicAdd(&hist[bb], 1u);
+      bins[j] = (uint16_t)bb;
+    }
+    __syncthreads();
+    // 3. threshold bin: thread t owns bins 4095 - 8t .. 4088 - 8t (descending)
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { c[j] = hist[TK_BINS - 1 - 8 * tid - j]; sum += c[j]; }
+    uint32_t incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -255,7 +270,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
     uint32_t before = 0;
     for (int w = 0; w < warp; ++w) before += wtot[w];
     incl += before;
-    const uint32_t excl = incl - s;
+    const uint32_t excl = incl - sum;
     if (excl < (uint32_t)topk && incl >= (uint32_t)topk) {
       uint32_t above = excl;
 #pragma unroll
@@ -273,60 +288,109 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
     T = bcast[0];
     remaining = topk - bcast[1];
     const int cntT = bcast[2];
-    if (cntT == remaining) {
-      emit_where([&](int i) { return bin_of(vals[i]) >= T; }, nv, out, topk, wsum);
-      return;
-    }
-    if (cntT > TK_CAND) fast = false;
-  }
-  if (fast) {
-    // candidates of bin T, then the remaining-th largest (score desc, index asc)
-    for (int j = tid; j < nv; j += TOPK_THREADS) {
-      const float v = vals[j];
-      if (bin_of(v) == T) cand[atomicAdd(&n_cand, 1)] = composite(v, j);
-    }
-    __syncthreads();
-    const int C = n_cand;
-    if (C <= TOPK_THREADS) {
-      if (tid < C) {
-        const uint64_t me = cand[tid];
-        int rank = 0;
-        for (int j = 0; j < C; ++j) rank += cand[j] > me;
-        if (rank == remaining - 1) thr_comp = me;
-      }
-    } else {
-      int P = 1;
-      while (P < C) P <<= 1;
-      for (int j = C + tid; j < P; j += TOPK_THREADS) cand[j] = 0ull;
-      __syncthreads();
-      for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          for (int i = tid; i < P; i += TOPK_THREADS) {
-            const int jx = i ^ stride;
-            if (jx > i) {
-              const bool desc = (i & size) == 0;
-              const uint64_t a = cand[i], c2 = cand[jx];
-              if ((a < c2) == desc) { cand[i] = c2; cand[jx] = a; }
-            }
-          }
-          __syncthreads();
+    take_all = (cntT == remaining);
+    if (!take_all && cntT > TK_CAND) fast = false;
+    if (fast && !take_all) {
+      // candidates of bin T (re-read from global), ranked by (score desc, index asc)
+      const int n8 = (nv + 7) >> 3;
+      for (int j8 = tid; j8 < n8; j8 += TOPK_THREADS) {
+        const uint4 bv = reinterpret_cast<const uint4*>(bins)[j8];
+        const uint32_t wds[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int i = 8 * j8 + q;
+          const uint32_t bi = (wds[q >> 1] >> (16 * (q & 1))) & 0xffffu;
+          if (i < nv && (int)bi == T) cand[atomicAdd(&n_cand, 1)] = composite(__ldg(srow + i), i);
         }
       }
-      if (tid == 0) thr_comp = cand[remaining - 1];
+      __syncthreads();
+      const int C = n_cand;
+      if (C <= TOPK_THREADS) {
+        if (tid < C) {
+          const uint64_t me = cand[tid];
+          int rank = 0;
+          for (int j = 0; j < C; ++j) rank += cand[j] > me;
+          if (rank < remaining) {
+            const int i = (int)(0xffffffffu - (uint32_t)me);
+            atomicOr(&selbits[i >> 5], 1u << (i & 31));
+          }
+        }
+      } else {
+        int P = 1;
+        while (P < C) P <<= 1;
+        for (int j = C + tid; j < P; j += TOPK_THREADS) cand[j] = 0ull;
+        __syncthreads();
+        for (int size = 2; size <= P; size <<= 1) {
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = tid; i < P; i += TOPK_THREADS) {
+              const int jx = i ^ stride;
+              if (jx > i) {
+                const bool desc = (i & size) == 0;
+                const uint64_t a = cand[i], c2 = cand[jx];
+                if ((a < c2) == desc) { cand[i] = c2; cand[jx] = a; }
+              }
+            }
+            __syncthreads();
+          }
+        }
+        for (int j = tid; j < remaining; j += TOPK_THREADS) {
+          const int i = (int)(0xffffffffu - (uint32_t)cand[j]);
+          atomicOr(&selbits[i >> 5], 1u << (i & 31));
+        }
+      }
+      __syncthreads();
     }
+  }
+  if (fast) {
+    // 4. count per warp segment, then write in ascending index order (8 bins per lane per step)
+    const int seg = ((nv + TOPK_WARPS - 1) / TOPK_WARPS + 255) & ~255;
+    const int lo_i = warp * seg, hi_i = min(nv, lo_i + seg);
+    auto sel_mask = [&](int base) -> uint32_t {   // 8-bit selection mask of elements base .. base+7
+      if (base >= hi_i) return 0u;
+      const uint4 bv = reinterpret_cast<const uint4*>(bins)[base >> 3];
+      const uint32_t wds[4] = {bv.x, bv.y, bv.z, bv.w};
+      uint32_t msk = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int i = base + q;
+        const int bi = (int)((wds[q >> 1] >> (16 * (q & 1))) & 0xffffu);
+        bool sel = bi > T || (bi == T && (take_all || ((selbits[i >> 5] >> (i & 31)) & 1u)));
+        if (i >= hi_i) sel = false;
+        msk |= (uint32_t)sel << q;
+      }
+      return msk;
+    };
+    int cnt = 0;
+    for (int base = lo_i; base < hi_i; base += 256) cnt += __popc(sel_mask(base + 8 * lane));
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) wsum[warp] = cnt;
     __syncthreads();
-    const uint64_t tc = thr_comp;
-    emit_where([&](int i) {
-      const float v = vals[i];
-      const int bi = bin_of(v);
-      return bi > T || (bi == T && composite(v, i) >= tc);
-    }, nv, out, topk, wsum);
+    int run = 0;
+    for (int w = 0; w < warp; ++w) run += wsum[w];
+    for (int base = lo_i; base < hi_i; base += 256) {
+      uint32_t msk = sel_mask(base + 8 * lane);
+      const int c8 = __popc(msk);
+      int incl2 = c8;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl2, o);
+        if (lane >= o) incl2 += v;
+      }
+      int pos = run + incl2 - c8;
+      while (msk) {
+        const int q = __ffs(msk) - 1;
+        if (pos < topk) out[pos] = base + 8 * lane + q;
+        ++pos;
+        msk &= msk - 1;
+      }
+      run += __shfl_sync(0xffffffffu, incl2, 31);
+    }
     return;
   }
-  // exact radix select over order-preserving keys (degenerate value ranges)
+  // exact radix select over order-preserving keys (degenerate value ranges / crowded bins)
   __syncthreads();
-  uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
-  for (int j = tid; j < nv; j += TOPK_THREADS) keys[j] = float_key(vals[j]);
+  uint32_t* keys = dyn;
+  for (int j = tid; j < nv; j += TOPK_THREADS) keys[j] = float_key(__ldcs(srow + j));
   __syncthreads();
   const RadixResult rr = radix_select(keys, nv, topk, hist, bcast);
   emit_selection(keys, nv, rr, out, topk, wsum);
@@ -342,7 +406,7 @@ cslc_status launch_topk_rows(const float* scores, int rows_in_buf, int row_begin
   cudaGetDevice(&dev);
   if (configured_for != dev) {
     cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         192 * 1024);
+                         TK_MAXN * 4);
     configured_for = dev;
   }
   dim3 grid(row_end - row_begin, B);

@@ -119,7 +119,8 @@ cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z,
  *   idx    [B, L, topk] int32
  *   ws     workspace of csa_indexer_topk_workspace_bytes() bytes (may be NULL
  *          when that is 0).
- * Requires d_I == 64, 1 <= H_I <= 16, 1 <= topk <= 2048, q_pos0 >= 0.
+ * Requires d_I == 64, 1 <= H_I <= 16, 1 <= topk <= 2048, q_pos0 >= 0,
+ * Nc <= 45056 (a row of scores is selected in shared memory).
  */
 size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given);
 cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w,
