@@ -43,9 +43,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Order-preserving map of an fp32 to uint32: a > b  <=>  key(a) > key(b).
+// Order-preserving map of an fp32 score to uint32: a > b  <=>  key(a) > key(b);
+// -0 maps to the key of +0 (the two compare equal as values, so they tie).
 __device__ __forceinline__ uint32_t float_key(float f) {
-  uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -5,19 +5,21 @@
 // Rule: the min(k, n_vis) visible entries with the largest fp32 score, ties
 // to the smaller entry index, emitted in ascending index order, -1 padded.
 //
-// One CTA per query row. The row's visible scores are mapped to
-// order-preserving uint32 keys in shared memory, the k-th largest key is found
-// by a most-significant-digit radix select (8-bit digits, per-warp histograms
-// with warp-aggregated shared-memory atomics; it stops early once every key
-// sharing the chosen prefix is known to be selected), and the selection is
-// compacted in index order with warp ballots: one pass counts per warp
-// segment, one writes. Ties at the threshold take the smallest indices.
+// Each row is selected by one small CTA. The fast path (below, at
+// topk_rows_kernel) bins the scores into a value-range histogram, ranks only
+// the scores near the bin that holds the k-th largest one, and compacts the
+// selection in index order. Rows it cannot take map their scores to
+// order-preserving uint32 keys and find the k-th largest key by a
+// most-significant-digit radix select (8-bit digits, per-warp histograms; it
+// stops early once every key sharing the chosen prefix is known to be
+// selected); the selection is then compacted in index order with warp
+// ballots. Ties at the threshold take the smallest indices.
 
 #include "common.cuh"
 
 namespace cslc {
 
-constexpr int TOPK_THREADS = 512;
+constexpr int TOPK_THREADS = 128;
 constexpr int TOPK_WARPS = TOPK_THREADS / 32;
 
 struct RadixResult {
@@ -26,10 +28,10 @@ struct RadixResult {
   int take_all;    // every key matching the prefix is selected
 };
 
-// Block-wide radix select of the `k`-th largest key among keys[0..n).
+// Block-wide radix select of the `k`-th largest key among key_of(0..n-1).
 // Requires blockDim.x == TOPK_THREADS and k <= n. hist: TOPK_WARPS * 256 words.
-__device__ RadixResult radix_select(const uint32_t* keys, int n, int k, uint32_t* hist,
-                                    int* bcast) {
+template <class KeyFn>
+__device__ RadixResult radix_select(KeyFn key_of, int n, int k, uint32_t* hist, int* bcast) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   RadixResult r{0u, 0u, k, 0};
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -38,7 +40,7 @@ __device__ RadixResult radix_select(const uint32_t* keys, int n, int k, uint32_t
     __syncthreads();
     uint32_t* hw = hist + warp * 256;
     for (int i = tid; i < n; i += TOPK_THREADS) {
-      const uint32_t key = keys[i];
+      const uint32_t key = key_of(i);
       if ((key & r.mask) == r.prefix) {
         const uint32_t d = (key >> shift) & 255u;
         const unsigned peers = __match_any_sync(__activemask(), d);
@@ -46,10 +48,10 @@ __device__ RadixResult radix_select(const uint32_t* keys, int n, int k, uint32_t
       }
     }
     __syncthreads();
-    if (tid < 256) {
+    for (int d = tid; d < 256; d += TOPK_THREADS) {
       uint32_t s = 0;
-      for (int w = 0; w < TOPK_WARPS; ++w) s += hist[w * 256 + tid];
-      hist[tid] = s;   // warp 0's copy becomes the total (read below only after the sync)
+      for (int w = 0; w < TOPK_WARPS; ++w) s += hist[w * 256 + d];
+      hist[d] = s;   // warp 0's copy becomes the total (read below only after the sync)
     }
     __syncthreads();
     if (warp == 0) {
@@ -91,10 +93,11 @@ __device__ RadixResult radix_select(const uint32_t* keys, int n, int k, uint32_t
   return r;
 }
 
-// Compacts the selected indices of keys[0..n) into out[] in ascending index
+// Compacts the selected indices of key_of(0..n-1) into out[] in ascending index
 // order (exactly k of them). wsum: 2 * TOPK_WARPS ints of shared memory.
-__device__ void emit_selection(const uint32_t* keys, int n, const RadixResult& r, int32_t* out,
-                               int k, int* wsum) {
+template <class KeyFn>
+__device__ void emit_selection(KeyFn key_of, int n, const RadixResult& r, int32_t* out, int k,
+                               int* wsum) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = ((n + TOPK_WARPS - 1) / TOPK_WARPS + 31) & ~31;
   const int lo = warp * seg, hi = min(n, lo + seg);
@@ -103,7 +106,7 @@ __device__ void emit_selection(const uint32_t* keys, int n, const RadixResult& r
   int n_eq = 0, n_gt = 0;
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
-    const uint32_t key = i < hi ? (keys[i] & r.mask) : 0u;
+    const uint32_t key = i < hi ? (key_of(i) & r.mask) : 0u;
     const bool valid = i < hi;
     n_eq += __popc(__ballot_sync(0xffffffffu, valid && key == r.prefix));
     n_gt += __popc(__ballot_sync(0xffffffffu, valid && key > r.prefix));
@@ -126,7 +129,7 @@ __device__ void emit_selection(const uint32_t* keys, int n, const RadixResult& r
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
     const bool valid = i < hi;
-    const uint32_t key = valid ? (keys[i] & r.mask) : 0u;
+    const uint32_t key = valid ? (key_of(i) & r.mask) : 0u;
     const bool is_eq = valid && key == r.prefix;
     const unsigned eq_mask = __ballot_sync(0xffffffffu, is_eq);
     const int eq_rank = eq_run + __popc(eq_mask & lt);
@@ -139,45 +142,77 @@ __device__ void emit_selection(const uint32_t* keys, int n, const RadixResult& r
   }
 }
 
-constexpr int TK_BINS = 4096;   // value-range histogram bins (shares storage with the radix histogram)
-constexpr int TK_CAND = 2048;   // threshold-bin candidates handled in shared memory
+constexpr int TK_SLICE = 4 * TOPK_THREADS;   // entries per slice
+constexpr int TK_BATCH = 8;                  // 16-byte loads per thread in flight
+constexpr int TK_BINS = 2048;                // value-range histogram bins
+constexpr int TK_CAND = 512;                 // keys near the threshold ranked in shared memory
+constexpr float TK_MAGIC = 12582912.f;       // 1.5 * 2^23: adding it leaves round(x) in the low mantissa bits
+static_assert(TK_BINS >= TOPK_WARPS * 256, "the value histogram doubles as the radix histograms");
+static_assert(TK_BINS == 16 * TOPK_THREADS, "the threshold scan gives each thread 16 bins");
 
 __device__ __forceinline__ uint64_t composite(float v, int i) {
   return ((uint64_t)float_key(v) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
 }
 
-// One CTA per query row.
-// Fast path (touches each score a few times with cheap work):
-//   1. each thread loads its scores with all loads in flight; one of them per
-//      thread, spread over the row, fixes a value range [lo, hi];
-//   2. one pass over those registers bins every score into 4096 equal
-//      bins of that range (scores outside clamp to the edge bins, which keeps
-//      the binning monotone), adds it to a shared histogram and keeps its
-//      16-bit bin in shared memory;
-//   3. the bin T holding the k-th largest score is found by a block scan; all
-//      scores in higher bins are selected; when bin T must be split, its
-//      scores are re-read and ranked exactly by (score desc, index asc) and the
-//      chosen ones are marked in a bitmap;
-//   4. two passes over the 16-bit bins (eight per 16-byte read) count the
-//      selection per warp segment and then write the indices in ascending order.
-// Rows whose sampled range is degenerate, or whose threshold bin is too
-// crowded, take the exact 8-bit radix select over order-preserving keys.
-constexpr int TK_MAXN = 45056;   // longest row (entries) the shared memory holds
-constexpr int TK_REG = 8;        // float4 loads per thread held in registers (power of two)
+__device__ __forceinline__ int tk_bin(float v, float lo, float bscale) {
+  const float t = fminf(fmaxf(fmaf(v - lo, bscale, TK_MAGIC), TK_MAGIC), TK_MAGIC + (float)(TK_BINS - 1));
+  return (int)(__float_as_uint(t) & (uint32_t)(TK_BINS - 1));
+}
 
-__global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
+// Block-wide exclusive scan of one int per thread; also returns the total.
+__device__ __forceinline__ int tk_block_excl_scan(int v, int* wtot, int& total) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < TOPK_WARPS; ++w) {
+    const int t = wtot[w];
+    before += w < warp ? t : 0;
+    total += t;
+  }
+  return before + incl - v;
+}
+
+// One CTA of TOPK_THREADS threads per query row; many rows per SM run side by
+// side. The row is read in slices of TK_SLICE entries (thread t reads entries
+// 4t..4t+3 of each slice with one 16-byte load); entries past n_vis read NaN.
+// Fast path:
+//   A. one pass counts every score in a 2048-bin histogram over a value range
+//      [lo, hi] taken from one score per thread of the first loads (scores
+//      outside clamp to the edge bins, so the binning stays monotone);
+//   B. a block scan of the histogram finds the bin T holding the k-th largest
+//      score; fp32 bounds lo_T < hi_T are put one and a half bins either side
+//      of T. A second pass (the row is still in L2) marks every score above
+//      hi_T in a 4-bit mask per four entries (shared memory), counts them
+//      exactly and collects the (score, index) keys in (lo_T, hi_T]. With fewer
+//      than k above hi_T and at least k above lo_T, the k-th key is among the
+//      collected ones: ranking them by (score desc, index asc) picks the
+//      remaining ones, whose bits are then set;
+//   C. the mask words are counted per thread, scanned across the block, and
+//      each thread writes the indices of its set bits in ascending order.
+// Rows for which a check fails (degenerate sampled range, too many collected
+// keys, bounds that miss the k-th score, e.g. through NaN scores) take the
+// exact 8-bit radix select over order-preserving keys read from the row.
+__global__ void __launch_bounds__(TOPK_THREADS, 8) topk_rows_kernel(
     const float* __restrict__ scores, int rows_in_buf, int row_begin, int L, int Nc, int m,
     int q_pos0, int topk, int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) uint32_t dyn[];          // n words: bins (fast) or keys (fallback)
-  __shared__ uint32_t hist[TK_BINS];
+  extern __shared__ __align__(16) uint32_t nibw[];   // 4-bit masks: entries 16w..16w+15 in word w
+  uint8_t* nib = reinterpret_cast<uint8_t*>(nibw);
+  __shared__ __align__(16) uint32_t hist[TK_BINS];
   __shared__ uint64_t cand[TK_CAND];
-  __shared__ uint32_t selbits[TK_MAXN / 32];
   __shared__ float red[2][TOPK_WARPS];
-  __shared__ uint32_t wtot[TOPK_WARPS];
+  __shared__ int wtot[TOPK_WARPS];
   __shared__ int bcast[4];
   __shared__ int wsum[2 * TOPK_WARPS];
   __shared__ int n_cand;
-  __shared__ uint64_t thr_comp;
   const int r = row_begin + blockIdx.x;
   const int b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -188,131 +223,139 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
     return;
   }
   const float* srow = scores + ((size_t)b * rows_in_buf + (r - row_begin)) * (size_t)Nc;
-  uint16_t* bins = reinterpret_cast<uint16_t*>(dyn);
-  for (int x = tid; x < TK_BINS; x += TOPK_THREADS) hist[x] = 0;
-  for (int x = tid; x < (nv + 31) / 32; x += TOPK_THREADS) selbits[x] = 0;
+  const int n_sl = (nv + TK_SLICE - 1) / TK_SLICE;
+#pragma unroll
+  for (int j = 0; j < TK_BINS / (4 * TOPK_THREADS); ++j)
+    reinterpret_cast<uint4*>(hist)[j * TOPK_THREADS + tid] = make_uint4(0u, 0u, 0u, 0u);
   if (tid == 0) n_cand = 0;
-  // 1. the row's first TK_REG * 4 * TOPK_THREADS scores go to registers with all
-  //    loads in flight at once; one of them per thread (spread over the row)
-  //    samples the value range
-  const bool vec = (Nc & 3) == 0;
-  const int n4 = vec ? (nv >> 2) : 0;
-  float4 rv[TK_REG];
-#pragma unroll
-  for (int i = 0; i < TK_REG; ++i) {
-    const int j = tid + i * TOPK_THREADS;
-    rv[i] = j < n4 ? __ldcs(reinterpret_cast<const float4*>(srow) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  {
-    const int si = tid & (TK_REG - 1);
-    const int sj = tid + si * TOPK_THREADS;
-    float v;
-    if (vec && sj < n4) {
-      v = rv[0].x;
-#pragma unroll
-      for (int i = 1; i < TK_REG; ++i) if (i == si) v = rv[i].x;
-    } else {
-      v = __ldg(srow + (int)(((long long)tid * nv) / TOPK_THREADS));
+  const bool vec = (Nc & 3) == 0;   // rows start 16-byte aligned
+  auto load4 = [&](int e, bool last_use) -> float4 {   // entries e..e+3, NaN past the row
+    if (vec && e + 4 <= nv) {
+      const float4* p = reinterpret_cast<const float4*>(srow + e);
+      return last_use ? __ldcs(p) : __ldg(p);
     }
-    float vmin = v, vmax = v;
+    const float qnan = __int_as_float(0x7fc00000);
+    float4 f;
+    f.x = e + 0 < nv ? __ldg(srow + e + 0) : qnan;
+    f.y = e + 1 < nv ? __ldg(srow + e + 1) : qnan;
+    f.z = e + 2 < nv ? __ldg(srow + e + 2) : qnan;
+    f.w = e + 3 < nv ? __ldg(srow + e + 3) : qnan;
+    return f;
+  };
+  // A. histogram
+  bool fast = true;
+  float lo = 0.f, bscale = 0.f;
+  for (int s0 = 0; s0 < n_sl; s0 += TK_BATCH) {
+    float4 rv[TK_BATCH];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
-      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    for (int i = 0; i < TK_BATCH; ++i)
+      rv[i] = s0 + i < n_sl ? load4((s0 + i) * TK_SLICE + 4 * tid, false) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s0 == 0) {
+      // value range from one score per thread (fminf / fmaxf skip the NaN past the row)
+      const int si = tid & (TK_BATCH - 1);
+      float v = rv[0].x;
+#pragma unroll
+      for (int i = 1; i < TK_BATCH; ++i) v = (i == si && i < n_sl) ? rv[i].x : v;
+      float vmin = v, vmax = v;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      }
+      if (lane == 0) { red[0][warp] = vmin; red[1][warp] = vmax; }
+      __syncthreads();
+      lo = red[0][0];
+      float hi = red[1][0];
+#pragma unroll
+      for (int w = 1; w < TOPK_WARPS; ++w) { lo = fminf(lo, red[0][w]); hi = fmaxf(hi, red[1][w]); }
+      const float span = hi - lo;
+      bscale = (float)(TK_BINS - 1) / span;
+      fast = span > 0.f && isfinite(span) && isfinite(bscale);
     }
-    if (lane == 0) { red[0][warp] = vmin; red[1][warp] = vmax; }
-  }
-  __syncthreads();
-  float lo = red[0][0], hi = red[1][0];
-  for (int w = 1; w < TOPK_WARPS; ++w) { lo = fminf(lo, red[0][w]); hi = fmaxf(hi, red[1][w]); }
-  const float span = hi - lo;
-  bool fast = span > 0.f && isfinite(span) && nv <= TK_MAXN;
-  const float bscale = fast ? ((float)TK_BINS - 0.5f) / span : 0.f;
-  auto bin_of = [&](float v) { return min(TK_BINS - 1, max(0, (int)((v - lo) * bscale))); };
-  int T = 0, remaining = 0;
-  bool take_all = false;
-  if (fast) {
-    // 2. bin every score (registers / global -> histogram + 16-bit bins)
+    if (fast) {
 #pragma unroll
-    for (int i = 0; i < TK_REG; ++i) {
-      const int j = tid + i * TOPK_THREADS;
-      if (j < n4) {
-        const float4 v = rv[i];
-        const int b0 = bin_of(v.x), b1 = bin_of(v.y), b2 = bin_of(v.z), b3 = bin_of(v.w);
-        atomicAdd(&hist[b0], 1u); atomicAdd(&hist[b1], 1u); atomicAdd(&hist[b2], 1u); atomicAdd(&hist[b3], 1u);
-        reinterpret_cast<uint2*>(bins)[j] = make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+      for (int i = 0; i < TK_BATCH; ++i) {
+        const int e = (s0 + i) * TK_SLICE + 4 * tid;
+        if (e + 4 <= nv) {
+          atomicAdd(&hist[tk_bin(rv[i].x, lo, bscale)], 1u);
+          atomicAdd(&hist[tk_bin(rv[i].y, lo, bscale)], 1u);
+          atomicAdd(&hist[tk_bin(rv[i].z, lo, bscale)], 1u);
+          atomicAdd(&hist[tk_bin(rv[i].w, lo, bscale)], 1u);
+        } else if (e < nv) {
+          atomicAdd(&hist[tk_bin(rv[i].x, lo, bscale)], 1u);
+          if (e + 1 < nv) atomicAdd(&hist[tk_bin(rv[i].y, lo, bscale)], 1u);
+          if (e + 2 < nv) atomicAdd(&hist[tk_bin(rv[i].z, lo, bscale)], 1u);
+        }
       }
     }
-    for (int j = tid + TK_REG * TOPK_THREADS; j < n4; j += TOPK_THREADS) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(srow) + j);
-      const int b0 = bin_of(v.x), b1 = bin_of(v.y), b2 = bin_of(v.z), b3 = bin_of(v.w);
-      atomicAdd(&hist[b0], 1u); atomicAdd(&hist[b1], 1u); atomicAdd(&hist[b2], 1u); atomicAdd(&hist[b3], 1u);
-      reinterpret_cast<uint2*>(bins)[j] = make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
-    }
-    for (int j = (n4 << 2) + tid; j < nv; j += TOPK_THREADS) {
-      const int bb = bin_of(__ldcs(srow + j));
-      atomicAdd(&hist[bb], 1u);
-      bins[j] = (uint16_t)bb;
-    }
-    __syncthreads();
-    // 3. threshold bin: thread t owns bins 4095 - 8t .. 4088 - 8t (descending)
-    uint32_t c[8], sum = 0;
+  }
+  __syncthreads();
+  if (fast) {
+    // B1. threshold bin: thread t owns bins 2047 - 16t .. 2032 - 16t (descending)
+    uint32_t c[16], sum = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { c[j] = hist[TK_BINS - 1 - 8 * tid - j]; sum += c[j]; }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
+    for (int j = 0; j < 4; ++j) {
+      const uint4 h = reinterpret_cast<const uint4*>(hist)[(TK_BINS - 16 * (tid + 1)) / 4 + 3 - j];
+      c[4 * j + 0] = h.w; c[4 * j + 1] = h.z; c[4 * j + 2] = h.y; c[4 * j + 3] = h.x;
     }
-    if (lane == 31) wtot[warp] = incl;
-    __syncthreads();
-    uint32_t before = 0;
-    for (int w = 0; w < warp; ++w) before += wtot[w];
-    incl += before;
-    const uint32_t excl = incl - sum;
-    if (excl < (uint32_t)topk && incl >= (uint32_t)topk) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sum += c[j];
+    int tot_unused;
+    const uint32_t excl = (uint32_t)tk_block_excl_scan((int)sum, wtot, tot_unused);
+    if (excl < (uint32_t)topk && excl + sum >= (uint32_t)topk) {
       uint32_t above = excl;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (above + c[j] >= (uint32_t)topk) {
-          bcast[0] = TK_BINS - 1 - 8 * tid - j;
-          bcast[1] = (int)above;
-          bcast[2] = (int)c[j];
-          break;
-        }
+      for (int j = 0; j < 16; ++j) {
+        if (above + c[j] >= (uint32_t)topk) { bcast[0] = TK_BINS - 1 - 16 * tid - j; break; }
         above += c[j];
       }
     }
     __syncthreads();
-    T = bcast[0];
-    remaining = topk - bcast[1];
-    const int cntT = bcast[2];
-    take_all = (cntT == remaining);
-    if (!take_all && cntT > TK_CAND) fast = false;
-    if (fast && !take_all) {
-      // candidates of bin T (re-read from global), ranked by (score desc, index asc)
-      const int n8 = (nv + 7) >> 3;
-      for (int j8 = tid; j8 < n8; j8 += TOPK_THREADS) {
-        const uint4 bv = reinterpret_cast<const uint4*>(bins)[j8];
-        const uint32_t wds[4] = {bv.x, bv.y, bv.z, bv.w};
+    const int T = bcast[0];
+    const float lo_T = T == 0 ? -INFINITY : lo + ((float)T - 1.5f) / bscale;
+    const float hi_T = T == TK_BINS - 1 ? INFINITY : lo + ((float)T + 1.5f) / bscale;
+    // B2. masks of the scores above hi_T; keys in (lo_T, hi_T]
+    int above = 0;
+#pragma unroll 4
+    for (int sl = 0; sl < n_sl; ++sl) {
+      const int e = sl * TK_SLICE + 4 * tid;
+      const float4 f = load4(e, true);
+      const uint32_t mh = (uint32_t)(f.x > hi_T) | ((uint32_t)(f.y > hi_T) << 1) |
+                          ((uint32_t)(f.z > hi_T) << 2) | ((uint32_t)(f.w > hi_T) << 3);
+      const uint32_t ml = (uint32_t)(f.x > lo_T) | ((uint32_t)(f.y > lo_T) << 1) |
+                          ((uint32_t)(f.z > lo_T) << 2) | ((uint32_t)(f.w > lo_T) << 3);
+      nib[sl * TOPK_THREADS + tid] = (uint8_t)mh;
+      above += __popc(mh);
+      if (ml != mh) {
+        const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int i = 8 * j8 + q;
-          const uint32_t bi = (wds[q >> 1] >> (16 * (q & 1))) & 0xffffu;
-          if (i < nv && (int)bi == T) cand[atomicAdd(&n_cand, 1)] = composite(__ldg(srow + i), i);
+        for (int q = 0; q < 4; ++q) {
+          if (((ml ^ mh) >> q) & 1u) {
+            const int slot = atomicAdd(&n_cand, 1);
+            if (slot < TK_CAND) cand[slot] = composite(fv[q], e + q);
+          }
         }
       }
-      __syncthreads();
-      const int C = n_cand;
+    }
+    above = __reduce_add_sync(0xffffffffu, above);
+    if (lane == 0) wsum[warp] = above;
+    __syncthreads();
+    above = 0;
+#pragma unroll
+    for (int w = 0; w < TOPK_WARPS; ++w) above += wsum[w];
+    const int C = n_cand;
+    const int remaining = topk - above;
+    fast = above < topk && C >= remaining && C <= TK_CAND;
+    if (fast) {
+      // B3. the remaining largest collected keys join the selection
       if (C <= TOPK_THREADS) {
         if (tid < C) {
           const uint64_t me = cand[tid];
           int rank = 0;
           for (int j = 0; j < C; ++j) rank += cand[j] > me;
           if (rank < remaining) {
-            const int i = (int)(0xffffffffu - (uint32_t)me);
-            atomicOr(&selbits[i >> 5], 1u << (i & 31));
+            const int e = (int)(0xffffffffu - (uint32_t)me);
+            atomicOr(&nibw[e >> 4], 1u << (8 * ((e >> 2) & 3) + (e & 3)));
           }
         }
       } else {
@@ -334,81 +377,45 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_rows_kernel(
           }
         }
         for (int j = tid; j < remaining; j += TOPK_THREADS) {
-          const int i = (int)(0xffffffffu - (uint32_t)cand[j]);
-          atomicOr(&selbits[i >> 5], 1u << (i & 31));
+          const int e = (int)(0xffffffffu - (uint32_t)cand[j]);
+          atomicOr(&nibw[e >> 4], 1u << (8 * ((e >> 2) & 3) + (e & 3)));
         }
       }
       __syncthreads();
+      // C. write the set bits in ascending index order (16 entries per word)
+      const int n_words = n_sl * (TK_SLICE / 16);
+      const int wpt = (n_words + TOPK_THREADS - 1) / TOPK_THREADS;
+      const int w0 = min(tid * wpt, n_words), w1 = min(w0 + wpt, n_words);
+      int cnt = 0;
+      for (int w = w0; w < w1; ++w) cnt += __popc(nibw[w]);
+      int tot;
+      int pos = tk_block_excl_scan(cnt, wtot, tot);
+      for (int w = w0; w < w1; ++w) {
+        uint32_t x = nibw[w];
+        while (x) {
+          const int bit = __ffs(x) - 1;
+          if (pos < topk) out[pos] = 16 * w + 4 * (bit >> 3) + (bit & 7);
+          ++pos;
+          x &= x - 1;
+        }
+      }
+      return;
     }
   }
-  if (fast) {
-    // 4. count per warp segment, then write in ascending index order (8 bins per lane per step)
-    const int seg = ((nv + TOPK_WARPS - 1) / TOPK_WARPS + 255) & ~255;
-    const int lo_i = warp * seg, hi_i = min(nv, lo_i + seg);
-    auto sel_mask = [&](int base) -> uint32_t {   // 8-bit selection mask of elements base .. base+7
-      if (base >= hi_i) return 0u;
-      const uint4 bv = reinterpret_cast<const uint4*>(bins)[base >> 3];
-      const uint32_t wds[4] = {bv.x, bv.y, bv.z, bv.w};
-      uint32_t msk = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int i = base + q;
-        const int bi = (int)((wds[q >> 1] >> (16 * (q & 1))) & 0xffffu);
-        bool sel = bi > T || (bi == T && (take_all || ((selbits[i >> 5] >> (i & 31)) & 1u)));
-        if (i >= hi_i) sel = false;
-        msk |= (uint32_t)sel << q;
-      }
-      return msk;
-    };
-    int cnt = 0;
-    for (int base = lo_i; base < hi_i; base += 256) cnt += __popc(sel_mask(base + 8 * lane));
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (lane == 0) wsum[warp] = cnt;
-    __syncthreads();
-    int run = 0;
-    for (int w = 0; w < warp; ++w) run += wsum[w];
-    for (int base = lo_i; base < hi_i; base += 256) {
-      uint32_t msk = sel_mask(base + 8 * lane);
-      const int c8 = __popc(msk);
-      int incl2 = c8;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl2, o);
-        if (lane >= o) incl2 += v;
-      }
-      int pos = run + incl2 - c8;
-      while (msk) {
-        const int q = __ffs(msk) - 1;
-        if (pos < topk) out[pos] = base + 8 * lane + q;
-        ++pos;
-        msk &= msk - 1;
-      }
-      run += __shfl_sync(0xffffffffu, incl2, 31);
-    }
-    return;
-  }
-  // exact radix select over order-preserving keys (degenerate value ranges / crowded bins)
+  // exact radix select over order-preserving keys read from the row
   __syncthreads();
-  uint32_t* keys = dyn;
-  for (int j = tid; j < nv; j += TOPK_THREADS) keys[j] = float_key(__ldcs(srow + j));
-  __syncthreads();
-  const RadixResult rr = radix_select(keys, nv, topk, hist, bcast);
-  emit_selection(keys, nv, rr, out, topk, wsum);
+  auto key_of = [&](int i) { return float_key(__ldg(srow + i)); };
+  const RadixResult rr = radix_select(key_of, nv, topk, hist, bcast);
+  emit_selection(key_of, nv, rr, out, topk, wsum);
 }
 
 cslc_status launch_topk_rows(const float* scores, int rows_in_buf, int row_begin, int row_end,
                              int B, int L, int Nc, int m, int q_pos0, int topk, int32_t* idx,
                              cudaStream_t stream) {
   if (row_end <= row_begin || B == 0) return CSLC_OK;
-  const size_t smem = (size_t)Nc * 4;
-  static int configured_for = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_for != dev) {
-    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TK_MAXN * 4);
-    configured_for = dev;
-  }
+  // mask storage for the launch's longest row (rows see more entries as t grows)
+  const int nv_max = n_visible((long long)q_pos0 + row_end - 1, m, Nc);
+  const size_t smem = (size_t)((nv_max + TK_SLICE - 1) / TK_SLICE) * (TK_SLICE / 4);
   dim3 grid(row_end - row_begin, B);
   topk_rows_kernel<<<grid, TOPK_THREADS, smem, stream>>>(scores, rows_in_buf, row_begin, L, Nc, m,
                                                          q_pos0, topk, idx);

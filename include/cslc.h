@@ -110,7 +110,9 @@ cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z,
  * for the entries visible to query row t (absolute position q_pos0 + t),
  * computed with fp32 accumulation of bf16 products and stored fp32.
  * idx[b,t,:] = the min(topk, n_vis) visible entries with the largest S (ties
- * to the smaller entry index), in ascending index order, then -1 padding.
+ * to the smaller entry index; -0 and +0 tie), in ascending index order, then
+ * -1 padding. Scores may be +-inf; a row holding a NaN score gets some valid
+ * selection of distinct visible entries, not a defined one.
  *
  *   q_idx  [B, L, H_I, d_I] bf16     w [B, L, H_I] bf16     k_idx [B, Nc, d_I] bf16
  *   scores [B, L, Nc] fp32 or NULL.  When given, row t holds S for entries

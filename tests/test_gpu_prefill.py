@@ -127,18 +127,53 @@ def test_indexer_topk_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
         assert np.all(v < nv)
 
 
-@pytest.mark.parametrize("Nc,L,topk,q_pos0,ties", [
-    (1024, 4096, 128, 0, False), (16384, 300, 1024, 65000, False), (16384, 64, 2048, 65300, True),
-    (1000, 333, 1, 3000, True), (5000, 100, 1024, 19000, True),
-])
-def test_topk_on_given_scores_bitexact(C, Nc, L, topk, q_pos0, ties):
-    m = 4
-    s = W.rand_f32((1, L, Nc), seed=700 + Nc)
-    if ties:   # few distinct values: many exact ties at the threshold
+def _topk_scores(kind, L, Nc, seed):
+    """Seeded score rows shaped to reach each branch of the prefill top-k."""
+    s = W.rand_f32((1, L, Nc), seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    if kind == "ties":        # few distinct values: many exact ties at the threshold
         s = torch.round(s * 2) / 2
+    elif kind in ("crowd", "mid"):   # a dense cluster of distinct values at the threshold
+        n, step = (5000, 6e-8) if kind == "crowd" else (1500, 1.2e-7)
+        for t in range(L):
+            cols = torch.randperm(Nc, generator=g)[:n]
+            s[0, t, cols] = 0.95 + torch.arange(n, dtype=torch.float32) * step
+    elif kind == "inf":       # non-finite scores
+        s[0, :, 3::97] = float("inf")
+        s[0, :, 5::89] = float("-inf")
+    elif kind == "outlier":   # extremes the sampled value range misses
+        s[0, :, 1001] = 1e30
+        s[0, :, 77] = -1e30
+    elif kind == "zeros":     # +0 and -0 tie at the threshold
+        z = torch.rand(s.shape, generator=g) < 0.95
+        sign0 = torch.where(torch.arange(Nc) % 2 == 0, 0.0, -0.0).expand_as(s)
+        s = torch.where(z, sign0, s + 0.1)
+    return s
+
+
+@pytest.mark.parametrize("Nc,L,topk,q_pos0,kind", [
+    (1024, 4096, 128, 0, "plain"), (16384, 300, 1024, 65000, "plain"),
+    (16384, 64, 2048, 65300, "ties"), (1000, 333, 1, 3000, "ties"), (5000, 100, 1024, 19000, "ties"),
+    (1001, 200, 100, 3000, "plain"), (16384, 24, 1024, 65536, "crowd"), (16384, 24, 1024, 65536, "mid"),
+    (8192, 40, 1024, 30000, "inf"), (8192, 40, 1024, 32768, "outlier"), (16384, 24, 1024, 65536, "zeros"),
+    (45056, 8, 1024, 4 * 45056, "plain"),
+])
+def test_topk_on_given_scores_bitexact(C, Nc, L, topk, q_pos0, kind):
+    m = 4
+    s = _topk_scores(kind, L, Nc, seed=700 + Nc)
     idx = C.csa_topk(dev(s), m=m, topk=topk, q_pos0=q_pos0)
     ref = O.topk_select(f64(s), m, topk, q_pos0)
     assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_rejects_unaligned_scores_pointer(C):
+    """Scores must start on a 16-byte boundary (the rows are read with 16-byte
+    loads); a view 4 bytes past one is refused before any launch."""
+    L, Nc = 8, 4096
+    flat = torch.zeros(L * Nc + 4, device="cuda")
+    view = flat[1:1 + L * Nc].view(1, L, Nc)
+    with pytest.raises(C.CslcError, match="ALIGN"):
+        C.csa_topk(view, m=4, topk=512, q_pos0=4 * Nc)
 
 
 def test_topk_all_equal_scores(C):
