@@ -59,15 +59,47 @@ static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
     REQUIRE(aligned16(p), CSLC_ERR_ALIGN, "%s: %s is not 16-byte aligned", __func__, #p); \
   } while (0)
 
-// scores rows are processed in blocks of this many rows when the caller does
-// not keep them: large enough that every indexer launch fills the GPU many
-// times over (the scores' HBM round trip costs far less than idle SMs)
+// When the caller does not keep the scores they are produced in blocks of
+// this many rows, two blocks in flight: the top-k of one block runs on an
+// auxiliary stream beside the indexer of the next, so neither launch's tail
+// leaves SMs idle.
 static int score_block_rows(int Nc) {
   const long long budget = 256ll << 20;   // bytes of scores per block
   long long rows = budget / ((long long)Nc * 4);
   rows = rows < 64 ? 64 : rows;
   rows = (rows / 64) * 64;
   return (int)rows;
+}
+
+// The auxiliary stream and its events, one set per host thread and device
+// (created on first use, kept for the life of the process).
+struct BlockOverlap {
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ready[2] = {nullptr, nullptr};   // scores of the block in buffer j written
+  cudaEvent_t freed[2] = {nullptr, nullptr};   // buffer j read by its top-k
+};
+
+static cslc_status block_overlap(BlockOverlap** out) {
+  constexpr int kMaxDevices = 64;
+  thread_local BlockOverlap sets[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: no usable current device");
+  BlockOverlap& o = sets[dev];
+  if (!o.aux) {
+    e = cudaStreamCreateWithFlags(&o.aux, cudaStreamNonBlocking);
+    for (int j = 0; j < 2 && e == cudaSuccess; ++j) {
+      e = cudaEventCreateWithFlags(&o.ready[j], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&o.freed[j], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {
+      o.aux = nullptr;
+      return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: stream/event creation: %s", cudaGetErrorString(e));
+    }
+  }
+  *out = &o;
+  return CSLC_OK;
 }
 
 }  // namespace cslc
@@ -121,7 +153,8 @@ size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, 
   if (scores_given || B <= 0 || L <= 0 || Nc <= 0) return 0;
   const int rows = score_block_rows(Nc);
   const int R = L < rows ? L : rows;
-  return (size_t)B * R * Nc * 4;
+  const int n_buf = L > R ? 2 : 1;
+  return (size_t)n_buf * B * R * Nc * 4;
 }
 
 cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w, const cslc_bf16* k_idx, int B,
@@ -151,15 +184,38 @@ cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w, const c
   }
   const int R = L < score_block_rows(Nc) ? L : score_block_rows(Nc);
   float* buf = static_cast<float*>(ws);
-  for (int r0 = 0; r0 < L; r0 += R) {
-    const int r1 = r0 + R < L ? r0 + R : L;
+  if (L <= R || Nc == 0) {
     if (Nc > 0) {
-      st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, r0, r1, buf, R, stream);
+      st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, buf, R, stream);
       if (st != CSLC_OK) return st;
     }
-    st = launch_topk_rows(buf, R, r0, r1, B, L, Nc, m, q_pos0, topk, idx, stream);
-    if (st != CSLC_OK) return st;
+    return launch_topk_rows(buf, R, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
   }
+  BlockOverlap* o = nullptr;
+  st = block_overlap(&o);
+  if (st != CSLC_OK) return st;
+  const size_t block_floats = (size_t)B * R * Nc;
+  int last = 0;
+  for (int i = 0, r0 = 0; r0 < L; ++i, r0 += R) {
+    const int r1 = r0 + R < L ? r0 + R : L;
+    const int j = i & 1;
+    float* bj = buf + j * block_floats;
+    cudaError_t e = i >= 2 ? cudaStreamWaitEvent(stream, o->freed[j], 0) : cudaSuccess;
+    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
+    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, r0, r1, bj, R, stream);
+    if (st != CSLC_OK) return st;
+    e = cudaEventRecord(o->ready[j], stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(o->aux, o->ready[j], 0);
+    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
+    st = launch_topk_rows(bj, R, r0, r1, B, L, Nc, m, q_pos0, topk, idx, o->aux);
+    if (st != CSLC_OK) return st;
+    e = cudaEventRecord(o->freed[j], o->aux);
+    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
+    last = j;
+  }
+  // join: `stream` continues after the last top-k (the auxiliary stream runs in order)
+  const cudaError_t e = cudaStreamWaitEvent(stream, o->freed[last], 0);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
   return CSLC_OK;
 }
 

@@ -117,7 +117,12 @@ cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z,
  *   q_idx  [B, L, H_I, d_I] bf16     w [B, L, H_I] bf16     k_idx [B, Nc, d_I] bf16
  *   scores [B, L, Nc] fp32 or NULL.  When given, row t holds S for entries
  *          0..n_vis(t)-1; entries from n_vis(t) on are left unspecified.
- *          When NULL the scores live only in the workspace, in row blocks.
+ *          When NULL the scores live only in the workspace, in blocks of
+ *          rows, two blocks in flight: the top-k of one block runs on an
+ *          internal stream (one per host thread and device) beside the
+ *          indexer of the next. All of it is ordered on `stream`: work queued
+ *          there before the call happens before, and work queued after the
+ *          call happens after (also under stream capture).
  *   idx    [B, L, topk] int32
  *   ws     workspace of csa_indexer_topk_workspace_bytes() bytes (may be NULL
  *          when that is 0).

@@ -127,6 +127,21 @@ def test_indexer_topk_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
         assert np.all(v < nv)
 
 
+def test_indexer_topk_blocks_in_flight(C):
+    """Without caller scores the rows go in blocks, two in flight on two
+    streams (three blocks here, so a buffer is reused): the selection equals
+    the one made from the full score tensor, which the oracle checks on
+    sampled rows."""
+    B, L, HI, m, topk, Nc = 2, 1500, 4, 4, 512, 45056
+    q_pos0 = m * Nc - L
+    assert C.indexer_topk_workspace_bytes(B, L, Nc, HI, topk) > B * L * Nc * 4 // 2
+    x, idx, idx_blocked, sc = _indexer_case(C, B, L, HI, m, topk, q_pos0, 37, Nc)
+    assert np.array_equal(idx_blocked, idx)
+    rows = sample_rows(L, 12, seed=37)
+    ref = O.topk_select(sc[:, rows], m, topk, q_pos0, rows=rows)
+    assert np.array_equal(idx[:, rows], ref)
+
+
 def _topk_scores(kind, L, Nc, seed):
     """Seeded score rows shaped to reach each branch of the prefill top-k."""
     s = W.rand_f32((1, L, Nc), seed=seed)
