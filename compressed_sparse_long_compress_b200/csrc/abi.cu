@@ -39,6 +39,7 @@ cslc_status launch_dense_attn(const uint16_t*, const uint16_t*, int, int, int, i
 size_t decode_workspace_bytes(const cslc_decode_layer*, int, int, int);
 int sparse_attn_sm100_read_error();
 int dense_attn_sm100_read_error();
+int indexer_sm100_read_error();
 size_t decode_topk_workspace_bytes(int, int, int);
 cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*, size_t, cudaStream_t);
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
@@ -121,6 +122,9 @@ cslc_status cslc_sync_status(cslc_stream_t stream) {
   const int code2 = dense_attn_sm100_read_error();
   if (code2 != 0)
     return set_error(CSLC_ERR_DEVICE_CHECK, "hca_dense_attn: a pipeline wait timed out (code %d)", code2);
+  const int code3 = indexer_sm100_read_error();
+  if (code3 != 0)
+    return set_error(CSLC_ERR_DEVICE_CHECK, "csa_indexer_topk: a pipeline wait timed out (code %d)", code3);
   return CSLC_OK;
 }
 

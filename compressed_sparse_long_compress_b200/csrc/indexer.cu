@@ -131,26 +131,30 @@ __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
           acc[nt][3] = fmaf(wb, fmaxf(d[3], 0.f), acc[nt][3]);
         }
       }
-      // store: entries past n_vis inside this tile get -inf; never past Nc
+      // store: entries past n_vis inside this tile get -inf; never past Nc. Pairs
+      // go out as one 8-byte store only when every row starts 8-byte aligned.
+      const bool pair_ok = (Nc & 1) == 0;
       float* sa = scores + ((size_t)b * rows_in_buf + (ra - row_begin)) * (size_t)Nc;
       float* sb = scores + ((size_t)b * rows_in_buf + (rb - row_begin)) * (size_t)Nc;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int col = e0 + nt * 8 + 2 * tq;
         if (ra < row_end && e0 < nva) {
-          if (col + 1 < Nc) {
+          if (pair_ok && col + 1 < Nc) {
             float2 v = make_float2(col < nva ? acc[nt][0] : -INFINITY, col + 1 < nva ? acc[nt][1] : -INFINITY);
             *reinterpret_cast<float2*>(sa + col) = v;
-          } else if (col < Nc) {
-            sa[col] = col < nva ? acc[nt][0] : -INFINITY;
+          } else {
+            if (col < Nc) sa[col] = col < nva ? acc[nt][0] : -INFINITY;
+            if (col + 1 < Nc) sa[col + 1] = col + 1 < nva ? acc[nt][1] : -INFINITY;
           }
         }
         if (rb < row_end && e0 < nvb) {
-          if (col + 1 < Nc) {
+          if (pair_ok && col + 1 < Nc) {
             float2 v = make_float2(col < nvb ? acc[nt][2] : -INFINITY, col + 1 < nvb ? acc[nt][3] : -INFINITY);
             *reinterpret_cast<float2*>(sb + col) = v;
-          } else if (col < Nc) {
-            sb[col] = col < nvb ? acc[nt][2] : -INFINITY;
+          } else {
+            if (col < Nc) sb[col] = col < nvb ? acc[nt][2] : -INFINITY;
+            if (col + 1 < Nc) sb[col + 1] = col + 1 < nvb ? acc[nt][3] : -INFINITY;
           }
         }
       }
@@ -164,10 +168,20 @@ size_t indexer_smem_bytes(int HI) {
   return (size_t)HI * IDX_ROWS * 128 + 2 * IDX_TILE * 128 + (size_t)IDX_ROWS * HI * 4;
 }
 
+bool indexer_sm100_supported(int HI);
+cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int B,
+                                 int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
+                                 float* scores, int rows_in_buf, cudaStream_t stream);
+
 cslc_status launch_indexer_scores(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
                                   int B, int L, int Nc, int HI, int m, int q_pos0, int row_begin,
                                   int row_end, float* scores, int rows_in_buf, cudaStream_t stream) {
   if (row_end <= row_begin || B == 0) return CSLC_OK;
+  // tensor-core path when whole TMA boxes fit the operands (256 query pairs,
+  // 128 entries); the mma.sync kernel below takes the rest
+  if (indexer_sm100_supported(HI) && (long long)B * L * HI >= 256 && (long long)B * Nc >= 128)
+    return launch_indexer_sm100(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores,
+                                rows_in_buf, stream);
   const size_t smem = indexer_smem_bytes(HI);
   static int configured_for = -1;
   int dev = 0;

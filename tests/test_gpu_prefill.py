@@ -104,6 +104,8 @@ def _indexer_case(C, B, L, HI, m, topk, q_pos0, wid, Nc=None):
     (1, 777, 16, 4, 100, 37, None),         # 16 indexer heads, query offset
     (1, 512, 1, 2, 300, 0, None),           # k above most rows' visible counts
     (1, 300, 8, 4, 2048, 4000, 1100),       # later queries of a longer sequence
+    (1, 700, 6, 4, 64, 0, None),            # H_I not a power of two (mma.sync kernel)
+    (1, 40, 4, 4, 16, 0, None),             # fewer than 256 query pairs (mma.sync kernel)
 ])
 def test_indexer_topk_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
     x, idx, idx_blocked, sc = _indexer_case(C, B, L, HI, m, topk, q_pos0, 31, Nc)
@@ -132,14 +134,21 @@ def test_indexer_topk_blocks_in_flight(C):
     streams (three blocks here, so a buffer is reused): the selection equals
     the one made from the full score tensor, which the oracle checks on
     sampled rows."""
-    B, L, HI, m, topk, Nc = 2, 1500, 4, 4, 512, 45056
+    B, L, HI, m, topk, Nc = 1, 3000, 4, 4, 512, 45056
     q_pos0 = m * Nc - L
-    assert C.indexer_topk_workspace_bytes(B, L, Nc, HI, topk) > B * L * Nc * 4 // 2
-    x, idx, idx_blocked, sc = _indexer_case(C, B, L, HI, m, topk, q_pos0, 37, Nc)
-    assert np.array_equal(idx_blocked, idx)
-    rows = sample_rows(L, 12, seed=37)
-    ref = O.topk_select(sc[:, rows], m, topk, q_pos0, rows=rows)
-    assert np.array_equal(idx[:, rows], ref)
+    block_bytes = C.indexer_topk_workspace_bytes(B, L, Nc, HI, topk) // 2
+    assert 0 < 2 * block_bytes < B * L * Nc * 4        # two buffers, each under half the rows
+    s = W.PrefillShape(B=B, L=L, H=16, m=m, HI=HI, topk=topk)
+    x = W.prefill_inputs(s, wid=41, with_indexer=True)
+    x["k_idx"] = W.randn_bf16((B, Nc, 64), W.seed_of(41, W.T_KIDX))
+    qi, w, k = dev(x["q_idx"]), dev(x["w"]), dev(x["k_idx"])
+    idx, scores = C.csa_indexer_topk(qi, w, k, m=m, topk=topk, q_pos0=q_pos0, scores=True)
+    idx_blocked, _ = C.csa_indexer_topk(qi, w, k, m=m, topk=topk, q_pos0=q_pos0)
+    assert torch.equal(idx_blocked, idx)
+    rows = sample_rows(L, 12, seed=41)
+    sc = f64(scores[:, torch.as_tensor(rows, device=scores.device)])
+    ref = O.topk_select(sc, m, topk, q_pos0, rows=rows)
+    assert np.array_equal(idx[:, torch.as_tensor(rows, device=idx.device)].cpu().numpy(), ref)
 
 
 def _topk_scores(kind, L, Nc, seed):
