@@ -415,6 +415,15 @@ def profile_case(name):
         idx = torch.empty(1, L, k, dtype=torch.int32, device=dev)
         for _ in range(2):
             C.csa_topk(scores, m=4, topk=k, q_pos0=4 * n_c, idx=idx)   # every row sees all entries
+    elif name == "indexer_L8192":
+        L, n_c, HI = 8192, 16384, 8
+        q_idx = W.randn_bf16((1, L, HI, 64), 5, device=dev)
+        w = W.randn_bf16((1, L, HI), 6, device=dev)
+        k_idx = W.randn_bf16((1, n_c, 64), 7, device=dev)
+        scores = torch.empty(1, L, n_c, device=dev)
+        idx = torch.empty(1, L, 1024, dtype=torch.int32, device=dev)
+        for _ in range(2):   # the last 8192 query rows of a 65536-token sequence
+            C.csa_indexer_topk(q_idx, w, k_idx, m=4, topk=1024, q_pos0=4 * n_c - L, scores=scores, idx=idx)
     else:
         raise SystemExit(f"unknown profile case {name}")
     torch.cuda.synchronize()
@@ -559,7 +568,7 @@ def main():
     ap.add_argument("--workload", default="csa_prefill", choices=list(W.WORKLOADS))
     ap.add_argument("--secondary", default="all", choices=["none", "all"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192"],
+    ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192", "indexer_L8192"],
                     help="run one small kernel case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:

@@ -19,8 +19,8 @@
 //              in shared memory), then the visible key tiles (TMA, 4 stages);
 //   warp 1     TMEM allocation and the single MMA-issuing thread (4 MMAs of
 //              K = 16 per tile, M = 128, N = 256);
-//   warps 2-9  epilogue: warp w reads TMEM lanes 32*(w%4).. (its entries) and
-//              one half of the columns, forms the scores of its rows and
+//   warps 2-17 epilogue: warp w reads TMEM lanes 32*(w%4).. (its entries) and
+//              one quarter of the columns, forms the scores of its rows and
 //              stores those of visible entries.
 // TMEM: two accumulators of 256 columns (tile j+1 is computed while tile j is
 // read out). All waits are time-bounded (abort + device error word).
@@ -35,13 +35,14 @@ __device__ int g_indexer_err = 0;
 
 namespace {
 
-constexpr int IX_THREADS = 320;
+constexpr int IX_THREADS = 576;
 constexpr int IX_PROD_WARP = 0;
 constexpr int IX_MMA_WARP = 1;
 constexpr int IX_EPI_WARP0 = 2;
-constexpr int IX_EPI_WARPS = 8;
+constexpr int IX_EPI_WARPS = 16;
 constexpr int IX_ET = 128;                       // entries per key tile (MMA M)
 constexpr int IX_NP = 256;                       // (token, head) pairs per query tile (MMA N)
+constexpr int IX_EPI_COLS = IX_NP / (IX_EPI_WARPS / 4);   // accumulator columns per epilogue warp
 constexpr int IX_KSTAGES = 4;
 constexpr int IX_K_BYTES = IX_ET * 128;          // 16 KB: 128 entries x 64 bf16
 constexpr int IX_Q_BYTES = IX_NP * 128;          // 32 KB: 256 pairs x 64 bf16
@@ -209,8 +210,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;                        // TMEM lanes 32*quad .. 32*quad+31
-    const int half = (warp - IX_EPI_WARP0) >> 2;      // columns 128*half .. 128*half+127
-    constexpr int RH = IX_NP / 2 / HI;                // rows per half
+    const int part = (warp - IX_EPI_WARP0) >> 2;      // columns IX_EPI_COLS*part ..
+    constexpr int RH = IX_EPI_COLS / HI;              // rows per part
     static_assert(32 % HI == 0, "a 32-column chunk holds whole rows");
     int rq = 0, kt = 0;
     bool ok = true;
@@ -221,9 +222,9 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       bool w_ok = true;
       if (lane == 0) w_ok = mbar_wait(&bars.q_full[qs], (uint32_t)((rq >> 1) & 1), abortp, errp, ERR_Q_FULL);
       if (!__shfl_sync(0xffffffffu, (int)w_ok, 0)) break;
-      const float4* wr = reinterpret_cast<const float4*>(w_s + qs * IX_NP + half * (IX_NP / 2));
-      const int* nvr = nv_s + qs * IX_NP + half * RH;
-      const int r0 = t0 + half * RH;                  // first row of this warp's half
+      const float4* wr = reinterpret_cast<const float4*>(w_s + qs * IX_NP + part * IX_EPI_COLS);
+      const int* nvr = nv_s + qs * IX_NP + part * RH;
+      const int r0 = t0 + part * RH;                  // first row of this warp's part
       float* out0 = scores + ((size_t)b * rows_in_buf + (r0 - row_begin)) * (size_t)Nc;
       for (int et = 0; et < n_et; ++et, ++kt) {
         const int ds = kt & 1;
@@ -232,25 +233,36 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
         if (!__shfl_sync(0xffffffffu, (int)d_ok, 0)) { ok = false; break; }
         tc_fence_after();
         const int e = et * IX_ET + quad * 32 + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ds * IX_NP + half * (IX_NP / 2);
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ds * IX_NP + part * IX_EPI_COLS;
+        // one 32-column chunk per TMEM wait; each score's head sum runs as two
+        // independent FMA chains
 #pragma unroll
-        for (int c = 0; c < (IX_NP / 2) / 32; ++c) {
+        for (int c = 0; c < IX_EPI_COLS / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
-          float wc[32];                               // weights of the chunk's 32 pairs
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const float4 f = wr[c * 8 + x];
-            wc[4 * x] = f.x; wc[4 * x + 1] = f.y; wc[4 * x + 2] = f.z; wc[4 * x + 3] = f.w;
-          }
           tmem_wait_ld();
 #pragma unroll
           for (int rr = 0; rr < 32 / HI; ++rr) {
             const int r = c * (32 / HI) + rr;
-            float s = 0.f;
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int h = 0; h < HI; ++h) s = fmaf(wc[rr * HI + h], fmaxf(__uint_as_float(v[rr * HI + h]), 0.f), s);
-            if (e < nvr[r]) out0[(size_t)r * Nc + e] = s;
+            for (int h4 = 0; h4 < (HI + 3) / 4; ++h4) {
+              const int p = rr * HI + 4 * h4;          // first pair of this group of 4 heads
+              float wq[4];
+              if (HI >= 4) {
+                const float4 f = wr[(c * 32 + p) / 4];
+                wq[0] = f.x; wq[1] = f.y; wq[2] = f.z; wq[3] = f.w;
+              } else {
+#pragma unroll
+                for (int q = 0; q < HI; ++q) wq[q] = reinterpret_cast<const float*>(wr)[c * 32 + p + q];
+              }
+#pragma unroll
+              for (int q = 0; q < (HI < 4 ? HI : 4); ++q) {
+                const float x = fmaxf(__uint_as_float(v[p + q]), 0.f);
+                if (q & 1) s1 = fmaf(wq[q], x, s1); else s0 = fmaf(wq[q], x, s0);
+              }
+            }
+            if (e < nvr[r]) out0[(size_t)r * Nc + e] = s0 + s1;
           }
         }
         tc_fence_before();
