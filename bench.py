@@ -75,6 +75,12 @@ class ClockSampler:
                  "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
+        # start timing only once the sampler is live (its first line is written)
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5.0:
+            if os.path.getsize(self.path) > 0 or self.proc.poll() is not None:
+                break
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
@@ -356,16 +362,24 @@ def time_e2e(wl, steps, world):
     return ms, sum(t.numel() * t.element_size() for t in ins), sum(t.numel() * t.element_size() for t in outs)
 
 
-def measure(name, C, args, world, rank, local, peaks, flush, with_e2e=True):
+def measure(name, C, args, world, rank, local, peaks, flush, with_e2e=True, min_timed_ms=0.0):
+    """min_timed_ms > 0 (secondary workloads only) raises the number of timed
+    steps until the timed region lasts about that long, so that the clock
+    sampler sees it; the headline workload times exactly args.steps."""
     device = torch.device("cuda", local)
     wl = make_workload(name, C, device, rank)
+    steps = args.steps
+    if min_timed_ms > 0:
+        probe, _ = time_device(wl, 2, 1, world, flush)
+        per = max(1e-3, max_over_ranks(max(probe), world))
+        steps = max(steps, int(min_timed_ms / per) + 1)
     with ClockSampler(local) as clk:
-        step_ms, kern_ms = time_device(wl, args.steps, args.warmup, world, flush)
+        step_ms, kern_ms = time_device(wl, steps, args.warmup, world, flush)
     clocks = clk.summary()
     ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
     kms = max_over_ranks(sum(kern_ms) / len(kern_ms), world)
     res = {"ms_per_step": ms, "kernel_ms": kms, "clocks": clocks, "roofline": wl.roofline(kms, peaks),
-           "gpu_launches": wl.launches * args.steps, "config": wl.config(), "units": wl.units}
+           "gpu_launches": wl.launches * steps, "config": wl.config(), "units": wl.units, "steps": steps}
     if wl.units > 1:
         res["value"] = world * wl.units / (ms * 1e-3)
         res["unit"] = "tokens/s"
@@ -436,11 +450,11 @@ def profile_case(name):
 # kernel source is the one that was measured.
 MEASURED_TRAFFIC = {
     "sparse": {"src": "sparse_attn_sm100.cu",
-               "sha256": "7ed05fe7c53211ef9cd7a027600107ce2aa0bc39fe9c860f85035ba4bc5adc08",
-               "bytes_per_token": (172.030464e6 + 101.147136e6) / 8192},
+               "sha256": "2101640d3670ed965063b862bfbaae2461b012a8f3dda0224ae2bfd2f24ec7a0",
+               "bytes_per_token": (172.144128e6 + 100.620032e6) / 8192},
     "dense": {"src": "dense_attn_sm100.cu",
-              "sha256": "dd8fec45b42bbc05b73ad2872a7b3c0f8d46e1ba28a96c6b8f4416c7f0dcf2ce",
-              "bytes_per_token": (1.074034e9 + 1.024294e9) / 65536},
+              "sha256": "ebe369f7ee47983d6c170cdce3599d7512ba0773663d881cf2c7ec2cc447afd7",
+              "bytes_per_token": (1.074352e9 + 1.022927e9) / 65536},
 }
 
 
@@ -562,7 +576,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="csa_prefill", choices=list(W.WORKLOADS))
@@ -592,9 +606,9 @@ def main():
     secondary = {}
     if args.secondary == "all" and args.workload == "csa_prefill":
         for name in ("hca_prefill", "hybrid_decode"):
-            r = measure(name, C, args, world, rank, local, peaks, flush, with_e2e=False)
+            r = measure(name, C, args, world, rank, local, peaks, flush, with_e2e=False, min_timed_ms=500.0)
             secondary[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "kernel_ms", "roofline",
-                                                  "clocks", "config")}
+                                                  "clocks", "config", "steps")}
             head["gpu_launches"] += r["gpu_launches"] * 0   # reported per workload below
             secondary[name]["gpu_launches"] = r["gpu_launches"]
 

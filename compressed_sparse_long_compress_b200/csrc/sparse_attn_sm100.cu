@@ -289,9 +289,14 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
             for (int h = 0; h < HT; ++h) v[h] = 0.f;
           }
         }
-        // j == 0 always takes the exact-max path (negm starts at +inf)
-        const bool slow = named_bar_or(3, SA_NSOFT, j == 0 || !(pmax <= SA_OVERFLOW) || !w);
-        if (*abortp) { ok = false; break; }
+        // j == 0 always takes the exact-max path (negm starts at +inf). A raised
+        // abort flag joins the vote, so that all softmax warps leave together
+        // (the named barriers stay matched).
+        bool slow = false;
+        if (named_bar_or(3, SA_NSOFT, j == 0 || !(pmax <= SA_OVERFLOW) || !w || *abortp != 0)) {
+          if (named_bar_or(3, SA_NSOFT, !w || *abortp != 0)) { ok = false; break; }
+          slow = true;
+        }
         if (slow) {
           // exact per-head maximum of this tile from S (still intact: the next
           // S into this buffer waits for this tile's p_full)
