@@ -30,7 +30,8 @@
 //               an L2-resident table gather at ~10 TB/s with cp.async but only
 //               ~2 TB/s with TMA tile::gather4.)
 //   warp 11     TMEM allocation and the single MMA-issuing thread.
-// TMEM: S^T double buffer (2 x 64 columns) + O^T double buffer (2 x 64).
+// TMEM: S^T triple buffer (3 x 64 columns) + O^T double buffer (2 x 64); PV runs
+// two tiles behind S^T so that the next S^T never waits for the softmax.
 // Every wait is time-bounded; a timeout raises a CTA-wide abort, records an
 // error code in a device word read by cslc_sync_status, and all roles leave.
 
@@ -58,6 +59,7 @@ constexpr int SA_P_BYTES = SA_TILE * 128; // 16 KB per P^T tile (64 heads bf16)
 constexpr int SA_Q_BYTES = SA_NP * 256;   // 16 KB (also the output staging)
 constexpr int SA_MAXK = 2048;
 constexpr float SA_OVERFLOW = 256.f;      // probabilities up to 2^8 are kept unrescaled
+constexpr uint32_t SA_O_COL = 192;        // TMEM: S^T buffers at columns 0, 64, 128; O^T at 192 and 256
 
 enum { ERR_KV_EMPTY = 1, ERR_TOK_FULL, ERR_KV_FULL, ERR_P_FULL, ERR_O_FREE, ERR_S_FULL,
        ERR_PV_DONE, ERR_O_FULL, ERR_Q_EMPTY, ERR_FINAL };
@@ -65,9 +67,9 @@ enum { ERR_KV_EMPTY = 1, ERR_TOK_FULL, ERR_KV_FULL, ERR_P_FULL, ERR_O_FREE, ERR_
 struct __align__(8) SaBars {
   uint64_t kv_full[SA_STAGES], kv_empty[SA_STAGES];
   uint64_t tok_full[2], q_empty[2];
-  uint64_t s_full[2];
+  uint64_t s_full[3];
   uint64_t p_full[2];
-  uint64_t pv_done;
+  uint64_t pv_done[2];   // per P^T buffer: its PV has completed
   uint64_t o_full[2], o_free[2];
   uint64_t final_bar;
 };
@@ -148,16 +150,16 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
     for (int s = 0; s < SA_STAGES; ++s) { mbar_init(&bars.kv_full[s], SA_NPROD); mbar_init(&bars.kv_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.tok_full[i], 1); mbar_init(&bars.q_empty[i], SA_NSOFT / 32);
-      mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], SA_NSOFT / 32);
       mbar_init(&bars.o_full[i], 1); mbar_init(&bars.o_free[i], SA_NSOFT / 32);
     }
-    mbar_init(&bars.pv_done, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&bars.s_full[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars.pv_done[i], 1);
     mbar_init(&bars.final_bar, 1);
     sm->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == SA_MMA_WARP) tmem_alloc(&sm->tmem_base, 256);
+  if (warp == SA_MMA_WARP) tmem_alloc(&sm->tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -263,11 +265,15 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
 #pragma unroll
       for (int h = 0; h < HT; ++h) negm[h] = INFINITY;
       for (int j = 0; j < nt; ++j) {
-        const int sb = s_it & 1, pb = p_it & 1;
+        const int sb = s_it % 3, pb = p_it & 1;
         // each warp waits for S on its own; a timeout anywhere raises the abort
         // flag, which every thread reads after the tile's CTA-wide barrier
         bool w = true;
-        if (lane == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
+        if (lane == 0) {
+          w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it / 3) & 1), abortp, errp, ERR_S_FULL);
+          // P^T buffer pb is free once the PV two tiles back has read it
+          if (w && p_it >= 2) w = mbar_wait(&bars.pv_done[pb], (uint32_t)(((p_it >> 1) - 1) & 1), abortp, errp, ERR_PV_DONE);
+        }
         w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
         const int slot = j * SA_TILE + row;
         const bool valid = slot < topk && is[slot] >= 0;
@@ -340,12 +346,13 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
           if (sm->any_rescale) {
             // O^T must be stable: the previous tile's PV has to be complete
             bool w2 = true;
-            if (tid == 0) w2 = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
+            if (tid == 0)
+              w2 = mbar_wait(&bars.pv_done[(p_it - 1) & 1], (uint32_t)(((p_it - 1) >> 1) & 1), abortp, errp, ERR_PV_DONE);
             ok = !named_bar_or(2, SA_NSOFT, !w2);
             if (!ok) break;
             tc_fence_after();
             uint32_t o[32];
-            const uint32_t oc = tmem + lane_off + 128 + ob * 64 + hh * 32;
+            const uint32_t oc = tmem + lane_off + SA_O_COL + ob * 64 + hh * 32;
             tmem_ld32(oc, o);
             tmem_wait_ld();
 #pragma unroll
@@ -401,7 +408,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
       if (hh * 32 < H) {
         uint32_t r[32];
         if (nt > 0) {
-          tmem_ld32(tmem + lane_off + 128 + ob * 64 + hh * 32, r);
+          tmem_ld32(tmem + lane_off + SA_O_COL + ob * 64 + hh * 32, r);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -441,14 +448,14 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         for (int k = 0; k < 8; ++k) {
           const uint64_t ad = smem_desc_sw128(e0 + k * 2048, SA_TILE * 128, 1024);
           const uint64_t bd = smem_desc_sw128(p0 + k * 2048, SA_TILE * 128, 1024);
-          mma_bf16(tmem + 128 + ob * 64, ad, bd, ID_O, (j_prev > 0 || k > 0) ? 1u : 0u);
+          mma_bf16(tmem + SA_O_COL + ob * 64, ad, bd, ID_O, (j_prev > 0 || k > 0) ? 1u : 0u);
         }
         mma_commit(&bars.kv_empty[stage_prev]);
-        mma_commit(&bars.pv_done);
+        mma_commit(&bars.pv_done[pb]);
         ++p_it;
         return true;
       };
-      // S^T[j+2] reuses S buffer j & 1; it is issued after PV(j), which waits
+      // S^T[j+3] reuses S buffer j % 3; it is issued after PV(j), which waits
       // for p_full(j), so the softmax has finished reading S^T[j] by then.
       int s_cnt = 0;
       for (long long g = blockIdx.x; g < n_tok && ok; g += gridDim.x, ++tk) {
@@ -460,9 +467,9 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
           break;
         }
         const uint32_t q0 = smem_u32(q_s + qb * SA_Q_BYTES);
-        int stage_prev = 0;
+        int stage_1 = 0, stage_2 = 0;   // stages of tiles j-1 and j-2
         for (int j = 0; j < nt; ++j) {
-          const int stage = kv_it % SA_STAGES, sb = s_cnt & 1;
+          const int stage = kv_it % SA_STAGES, sb = s_cnt % 3;
           if (!mbar_wait(&bars.kv_full[stage], (uint32_t)((kv_it / SA_STAGES) & 1), abortp, errp, ERR_KV_FULL)) { ok = false; break; }
           fence_proxy_async_smem();   // cp.async (generic proxy) writes -> tensor-core reads
           tc_fence_after();
@@ -475,12 +482,16 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
           }
           mma_commit(&bars.s_full[sb]);
           ++s_cnt;
-          if (j > 0 && !issue_pv(stage_prev, j - 1, ob)) { ok = false; break; }
-          stage_prev = stage;
+          // PV lags S by two tiles: S^T[j+1] needs only the gathered tile, not
+          // the softmax of tile j-1
+          if (j > 1 && !issue_pv(stage_2, j - 2, ob)) { ok = false; break; }
+          stage_2 = stage_1;
+          stage_1 = stage;
           ++kv_it;
         }
         if (!ok) break;
-        if (nt > 0 && !issue_pv(stage_prev, nt - 1, ob)) { ok = false; break; }
+        if (nt > 1 && !issue_pv(stage_2, nt - 2, ob)) { ok = false; break; }
+        if (nt > 0 && !issue_pv(stage_1, nt - 1, ob)) { ok = false; break; }
         mma_commit(&bars.o_full[ob]);
       }
       // every MMA issued so far has completed before TMEM is released
@@ -493,7 +504,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
   __syncthreads();
   if (warp == SA_MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
