@@ -13,8 +13,9 @@
 // columns inside one thread, and a warp's 32 lanes store 32 consecutive
 // entries of one score row (128-byte stores).
 //
-// CTA roles (persistent, one CTA per SM; query-row tiles in decreasing-work
-// order, dealt to the CTAs in a snake so that every CTA gets a similar load):
+// CTA roles (persistent, one CTA per SM; work items = a query-row tile and a
+// chunk of 16 key tiles, heavy rows first, dealt to the CTAs in a snake so that
+// every CTA gets a similar load):
 //   warp 0     producer: per row tile the Q tile (TMA) and the weights (fp32
 //              in shared memory), then the visible key tiles (TMA, 4 stages);
 //   warp 1     TMEM allocation and the single MMA-issuing thread (4 MMAs of
@@ -44,6 +45,7 @@ constexpr int IX_ET = 128;                       // entries per key tile (MMA M)
 constexpr int IX_NP = 256;                       // (token, head) pairs per query tile (MMA N)
 constexpr int IX_EPI_COLS = IX_NP / (IX_EPI_WARPS / 4);   // accumulator columns per epilogue warp
 constexpr int IX_KSTAGES = 4;
+constexpr int IX_CHUNK = 16;                     // key tiles per work item (2048 entries)
 constexpr int IX_K_BYTES = IX_ET * 128;          // 16 KB: 128 entries x 64 bf16
 constexpr int IX_Q_BYTES = IX_NP * 128;          // 32 KB: 256 pairs x 64 bf16
 
@@ -88,7 +90,11 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int rt_per_b = (row_end - row_begin + RT - 1) / RT;
-  const int n_rt = B * rt_per_b;
+  // work items: (query-row tile, chunk of IX_CHUNK key tiles), so that a block
+  // of rows with fewer row tiles than SMs still fills the GPU
+  const int et_max = (n_visible((long long)q_pos0 + row_end - 1, m, Nc) + IX_ET - 1) / IX_ET;
+  const int n_ch = max(1, (et_max + IX_CHUNK - 1) / IX_CHUNK);
+  const int n_items = B * rt_per_b * n_ch;
   const long long n_pairs = (long long)B * L * HI;
 
   if (tid == 0) {
@@ -111,17 +117,21 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
   volatile int* abortp = &sm->abort_flag;
   int* errp = &g_indexer_err;
 
-  // j-th row tile of this CTA (snake over rounds of gridDim.x) -> batch, first
-  // row, number of key tiles; false when the CTA has no more tiles
-  auto tile_of = [&](int j, int& b, int& t0, int& n_et) -> bool {
+  // j-th work item of this CTA (snake over rounds of gridDim.x) -> batch,
+  // first row, first key tile and number of key tiles (0: nothing visible in
+  // this chunk); false when the CTA has no more items
+  auto tile_of = [&](int j, int& b, int& t0, int& et0, int& n_et) -> bool {
     const int G = gridDim.x;
     const int i = j * G + ((j & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x);
-    if (i >= n_rt) return false;
-    const int rt = rt_per_b - 1 - i / B;           // heavy (late) rows first
-    b = i % B;
+    if (i >= n_items) return false;
+    const int rb = i / n_ch;
+    const int rt = rt_per_b - 1 - rb / B;          // heavy (late) rows first
+    b = rb % B;
     t0 = row_begin + rt * RT;
     const int t_last = min(t0 + RT, row_end) - 1;
-    n_et = (n_visible((long long)q_pos0 + t_last, m, Nc) + IX_ET - 1) / IX_ET;
+    const int n_all = (n_visible((long long)q_pos0 + t_last, m, Nc) + IX_ET - 1) / IX_ET;
+    et0 = (i % n_ch) * IX_CHUNK;
+    n_et = max(0, min(IX_CHUNK, n_all - et0));
     return true;
   };
 
@@ -130,8 +140,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
     if (lane == 0) { tma_prefetch_map(&tm_q); tma_prefetch_map(&tm_k); }
     int rq = 0, kt = 0;
     bool ok = true;
-    int b, t0, n_et;
-    for (int j = 0; ok && tile_of(j, b, t0, n_et); ++j) {
+    int b, t0, et0, n_et;
+    for (int j = 0; ok && tile_of(j, b, t0, et0, n_et); ++j) {
       if (n_et == 0) continue;
       const int qs = rq & 1;
       bool w_ok = true;
@@ -150,7 +160,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       if (lane == 0) {
         mbar_arrive_expect_tx(&bars.q_full[qs], IX_Q_BYTES);
         tma_load_2d(q_s + qs * IX_Q_BYTES, &tm_q, 0, (int)p0, &bars.q_full[qs]);
-        for (int et = 0; et < n_et; ++et, ++kt) {
+        for (int et = et0; et < et0 + n_et; ++et, ++kt) {
           const int ks = kt % IX_KSTAGES;
           if (kt >= IX_KSTAGES &&
               !mbar_wait(&bars.k_empty[ks], (uint32_t)((kt / IX_KSTAGES - 1) & 1), abortp, errp, ERR_K_EMPTY)) {
@@ -177,13 +187,13 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       constexpr uint32_t ID = idesc_bf16(IX_ET, IX_NP, false, false);
       int rq = 0, kt = 0;
       bool ok = true;
-      int b, t0, n_et;
-      for (int j = 0; ok && tile_of(j, b, t0, n_et); ++j) {
+      int b, t0, et0, n_et;
+      for (int j = 0; ok && tile_of(j, b, t0, et0, n_et); ++j) {
         if (n_et == 0) continue;
         const int qs = rq & 1;
         if (!mbar_wait(&bars.q_full[qs], (uint32_t)((rq >> 1) & 1), abortp, errp, ERR_Q_FULL)) break;
         const uint32_t q0 = smem_u32(q_s + qs * IX_Q_BYTES);
-        for (int et = 0; et < n_et; ++et, ++kt) {
+        for (int et = et0; et < et0 + n_et; ++et, ++kt) {
           const int ks = kt % IX_KSTAGES, ds = kt & 1;
           if (!mbar_wait(&bars.k_full[ks], (uint32_t)((kt / IX_KSTAGES) & 1), abortp, errp, ERR_K_FULL) ||
               (kt >= 2 && !mbar_wait(&bars.d_empty[ds], (uint32_t)(((kt >> 1) - 1) & 1), abortp, errp, ERR_D_EMPTY))) {
@@ -215,8 +225,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
     static_assert(32 % HI == 0, "a 32-column chunk holds whole rows");
     int rq = 0, kt = 0;
     bool ok = true;
-    int b, t0, n_et;
-    for (int j = 0; ok && tile_of(j, b, t0, n_et); ++j) {
+    int b, t0, et0, n_et;
+    for (int j = 0; ok && tile_of(j, b, t0, et0, n_et); ++j) {
       if (n_et == 0) continue;
       const int qs = rq & 1;
       bool w_ok = true;
@@ -226,7 +236,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       const int* nvr = nv_s + qs * IX_NP + part * RH;
       const int r0 = t0 + part * RH;                  // first row of this warp's part
       float* out0 = scores + ((size_t)b * rows_in_buf + (r0 - row_begin)) * (size_t)Nc;
-      for (int et = 0; et < n_et; ++et, ++kt) {
+      for (int et = et0; et < et0 + n_et; ++et, ++kt) {
         const int ds = kt & 1;
         bool d_ok = true;
         if (lane == 0) d_ok = mbar_wait(&bars.d_full[ds], (uint32_t)((kt >> 1) & 1), abortp, errp, ERR_D_FULL);
@@ -303,8 +313,10 @@ cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const
     configured_for = dev;
   }
   const int RT = IX_NP / HI;
-  const int n_rt = B * ((row_end - row_begin + RT - 1) / RT);
-  const int grid = n_rt < n_sm ? n_rt : n_sm;
+  const int et_max = (n_visible((long long)q_pos0 + row_end - 1, m, Nc) + IX_ET - 1) / IX_ET;
+  const int n_ch = et_max > IX_CHUNK ? (et_max + IX_CHUNK - 1) / IX_CHUNK : 1;
+  const int n_items = B * ((row_end - row_begin + RT - 1) / RT) * n_ch;
+  const int grid = n_items < n_sm ? n_items : n_sm;
   CUtensorMap tm_q, tm_k;
   if (!make_tmap_bf16_2d(&tm_q, q_idx, (uint64_t)B * L * HI, kDI, kDI * 2, IX_NP, 64) ||
       !make_tmap_bf16_2d(&tm_k, k_idx, (uint64_t)B * Nc, kDI, kDI * 2, IX_ET, 64))
