@@ -140,9 +140,22 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(wid: int, rank: int) -> int:
+    """Workload id whose seeded draws rank `rank` uses: every rank runs its own
+    independent sequence (weak scaling, no data-path exchange)."""
+    return wid + 10 * rank
+
+
+def job_value(units_per_rank: int, max_ms: float, world: int) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's step time."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 # ---------------------------------------------------------------- workloads
@@ -164,7 +177,7 @@ class CsaPrefill:
         wl = W.WORKLOADS["csa_prefill"]
         self.s = s = wl.csa
         self.C = C
-        self.x = W.prefill_inputs(s, wl.wid + 10 * rank, device=device)
+        self.x = W.prefill_inputs(s, rank_seed(wl.wid, rank), device=device)
         self.e = torch.empty(s.B, s.n_c, 128, dtype=torch.bfloat16, device=device)
         self.idx = torch.empty(s.B, s.L, s.topk, dtype=torch.int32, device=device)
         self.out = torch.empty_like(self.x["q"])
@@ -202,11 +215,7 @@ class CsaPrefill:
                 "algorithmic_flops_per_launch": self.flops_attn, "peak_source": peaks["source"] + " (burst)"}
 
     def config(self):
-        s = self.s
-        return {"workload": "csa_prefill: CSA prefill, batch 1, L=65536, m=4 -> 16384 entries, 64 heads x 128, "
-                            "indexer 8 x 64, top-k 1024, causal",
-                "global_batch": s.B, "seq_len": s.L, "heads": s.H, "head_dim": 128, "m": s.m, "topk": s.topk,
-                "indexer_heads": s.HI, "l2": "flushed between steps (512 MiB write)"}
+        return workload_config(self.name)
 
 
 class HcaPrefill:
@@ -216,7 +225,7 @@ class HcaPrefill:
         wl = W.WORKLOADS["hca_prefill"]
         self.s = s = wl.hca
         self.C = C
-        self.x = W.prefill_inputs(s, wl.wid + 10 * rank, device=device, with_indexer=False)
+        self.x = W.prefill_inputs(s, rank_seed(wl.wid, rank), device=device, with_indexer=False)
         self.e = torch.empty(s.B, s.n_c, 128, dtype=torch.bfloat16, device=device)
         self.out = torch.empty_like(self.x["q"])
         self.launches = 2
@@ -247,10 +256,7 @@ class HcaPrefill:
                 "peak_source": peaks["source"] + " (burst)"}
 
     def config(self):
-        s = self.s
-        return {"workload": "hca_prefill: HCA prefill, batch 1, L=1048576, m'=128 -> 8192 entries, 64 heads x 128, "
-                            "dense causal", "global_batch": s.B, "seq_len": s.L, "heads": s.H, "m_prime": s.m,
-                "l2": "inputs larger than L2 (q 16 GiB)"}
+        return workload_config(self.name)
 
 
 class Decode:
@@ -261,7 +267,7 @@ class Decode:
         self.C = C
         self.layers, self.bytes = [], 0
         for li, kind in enumerate(d.kinds):
-            x = W.decode_layer_inputs(d, li, wl.wid + 10 * rank, device=device)
+            x = W.decode_layer_inputs(d, li, rank_seed(wl.wid, rank), device=device)
             n = torch.full((d.B,), d.n_entries[li], dtype=torch.int32, device=device)
             nope, rope, sc = C.quantize_kv_mixed(x["kv"])
             del x["kv"]
@@ -298,10 +304,30 @@ class Decode:
                 "algorithmic_bytes_per_launch": self.bytes, "peak_source": peaks["source"]}
 
     def config(self):
-        d = self.d
-        return {"workload": f"{self.name}: " + W.WORKLOADS[self.name].description, "global_batch": d.B,
-                "layers": list(d.kinds), "entries": list(d.n_entries), "heads": d.H, "topk": d.topk,
+        return workload_config(self.name)
+
+
+def workload_config(name):
+    """The `config` object of a workload (no device needed; the reference arm
+    reports the same one)."""
+    wl = W.WORKLOADS[name]
+    if name == "csa_prefill":
+        s = wl.csa
+        return {"workload": "csa_prefill: CSA prefill, batch 1, L=65536, m=4 -> 16384 entries, 64 heads x 128, "
+                            "indexer 8 x 64, top-k 1024, causal",
+                "global_batch": s.B, "seq_len": s.L, "heads": s.H, "head_dim": 128, "m": s.m, "topk": s.topk,
+                "indexer_heads": s.HI, "l2": "flushed between steps (512 MiB write)"}
+    if name == "hca_prefill":
+        s = wl.hca
+        return {"workload": "hca_prefill: HCA prefill, batch 1, L=1048576, m'=128 -> 8192 entries, 64 heads x 128, "
+                            "dense causal", "global_batch": s.B, "seq_len": s.L, "heads": s.H, "m_prime": s.m,
+                "l2": "inputs larger than L2 (q 16 GiB)"}
+    if wl.decode is not None:
+        d = wl.decode
+        return {"workload": f"{name}: " + wl.description, "global_batch": d.B, "layers": list(d.kinds),
+                "entries": list(d.n_entries), "heads": d.H, "topk": d.topk,
                 "l2": "flushed between steps (512 MiB write)"}
+    return {"workload": f"{name}: " + wl.description}
 
 
 def make_workload(name, C, device, rank):
@@ -381,7 +407,7 @@ def measure(name, C, args, world, rank, local, peaks, flush, with_e2e=True, min_
     res = {"ms_per_step": ms, "kernel_ms": kms, "clocks": clocks, "roofline": wl.roofline(kms, peaks),
            "gpu_launches": wl.launches * steps, "config": wl.config(), "units": wl.units, "steps": steps}
     if wl.units > 1:
-        res["value"] = world * wl.units / (ms * 1e-3)
+        res["value"] = job_value(wl.units, ms, world)
         res["unit"] = "tokens/s"
         res["higher_is_better"] = True
     else:
@@ -391,7 +417,7 @@ def measure(name, C, args, world, rank, local, peaks, flush, with_e2e=True, min_
     if with_e2e:
         e_ms, bi, bo = time_e2e(wl, max(2, min(args.steps, 5)), world)
         e_ms = max_over_ranks(e_ms, world)
-        e_val = world * wl.units / (e_ms * 1e-3) if wl.units > 1 else e_ms * 1e3
+        e_val = job_value(wl.units, e_ms, world) if wl.units > 1 else e_ms * 1e3
         res["e2e"] = {"value": e_val, "unit": res["unit"], "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
     del wl
     torch.cuda.empty_cache()
@@ -567,7 +593,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": "CSA+HCA prefill tokens/s and 1M-ctx decode us/step; % of TC/HBM roofline",
             "value": v, "unit": unit, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": unit == "tokens/s", "dtype": "f64", "data": "synthetic",
-            "config": {"workload": name}, "vs_baseline": None,
+            "config": dict(workload_config(name), parallelism="rank 0 alone (host cores)"), "vs_baseline": None,
             "cpu_baseline": {"value": v, "unit": unit, "cores": blas_threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

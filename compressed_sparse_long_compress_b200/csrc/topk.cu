@@ -316,23 +316,33 @@ __global__ void __launch_bounds__(TOPK_THREADS, 8) topk_rows_kernel(
     const float hi_T = T == TK_BINS - 1 ? INFINITY : lo + ((float)T + 1.5f) / bscale;
     // B2. masks of the scores above hi_T; keys in (lo_T, hi_T]
     int above = 0;
-#pragma unroll 4
-    for (int sl = 0; sl < n_sl; ++sl) {
-      const int e = sl * TK_SLICE + 4 * tid;
-      const float4 f = load4(e, true);
-      const uint32_t mh = (uint32_t)(f.x > hi_T) | ((uint32_t)(f.y > hi_T) << 1) |
-                          ((uint32_t)(f.z > hi_T) << 2) | ((uint32_t)(f.w > hi_T) << 3);
-      const uint32_t ml = (uint32_t)(f.x > lo_T) | ((uint32_t)(f.y > lo_T) << 1) |
-                          ((uint32_t)(f.z > lo_T) << 2) | ((uint32_t)(f.w > lo_T) << 3);
-      nib[sl * TOPK_THREADS + tid] = (uint8_t)mh;
-      above += __popc(mh);
-      if (ml != mh) {
-        const float fv[4] = {f.x, f.y, f.z, f.w};
+    for (int s0 = 0; s0 < n_sl; s0 += TK_BATCH) {
+      // all of the batch's loads in flight before any is used
+      float4 rv[TK_BATCH];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (((ml ^ mh) >> q) & 1u) {
-            const int slot = atomicAdd(&n_cand, 1);
-            if (slot < TK_CAND) cand[slot] = composite(fv[q], e + q);
+      for (int i = 0; i < TK_BATCH; ++i)
+        rv[i] = s0 + i < n_sl ? load4((s0 + i) * TK_SLICE + 4 * tid, true)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < TK_BATCH; ++i) {
+        const int sl = s0 + i;
+        if (sl >= n_sl) break;
+        const int e = sl * TK_SLICE + 4 * tid;
+        const float4 f = rv[i];
+        const uint32_t mh = (uint32_t)(f.x > hi_T) | ((uint32_t)(f.y > hi_T) << 1) |
+                            ((uint32_t)(f.z > hi_T) << 2) | ((uint32_t)(f.w > hi_T) << 3);
+        const uint32_t ml = (uint32_t)(f.x > lo_T) | ((uint32_t)(f.y > lo_T) << 1) |
+                            ((uint32_t)(f.z > lo_T) << 2) | ((uint32_t)(f.w > lo_T) << 3);
+        nib[sl * TOPK_THREADS + tid] = (uint8_t)mh;
+        above += __popc(mh);
+        if (ml != mh) {
+          const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (((ml ^ mh) >> q) & 1u) {
+              const int slot = atomicAdd(&n_cand, 1);
+              if (slot < TK_CAND) cand[slot] = composite(fv[q], e + q);
+            }
           }
         }
       }
