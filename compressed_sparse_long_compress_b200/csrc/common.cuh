@@ -58,6 +58,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   int sz = valid ? 16 : 0;   // src-size 0 zero-fills the 16 destination bytes
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(sz));
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+  int sz = valid ? 4 : 0;    // src-size 0 zero-fills the 4 destination bytes
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(sz));
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 // Arrives on the mbarrier (without changing its expected count) once every
 // cp.async this thread issued so far has landed.

@@ -17,7 +17,7 @@
 //                          select on score key ++ reversed index, so ties go to
 //                          the smaller index), then a bitonic sort of the k
 //                          indices into ascending order
-//   decode_attn_kernel     split-K attention: each CTA dequantises 256 entries
+//   decode_attn_kernel     split-K attention: each CTA dequantises 128 entries
 //                          (e4m3 * scale -> bf16, RoPE half copied) into shared
 //                          memory and runs QK^T / softmax / PV for all heads
 //   decode_combine_kernel  merges the splits with their max / sum statistics
@@ -30,7 +30,7 @@ constexpr int DEC_CHUNK = 4096;      // entries per scores / select CTA
 constexpr int DEC_THREADS = 256;
 constexpr int HIST_BINS = 4096;      // top 12 bits of the score key
 constexpr int HIST_SHIFT = 20;
-constexpr int SPLIT = 256;           // entries per attention CTA
+constexpr int SPLIT = 128;           // entries per attention CTA
 constexpr int DTILE = 64;            // entries per attention tile
 constexpr int FIN_THREADS = 1024;
 constexpr int MAX_TOPK = 2048;
@@ -355,8 +355,11 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
     const int32_t* __restrict__ idx, int topk, int H, float scale_log2, int splits,
     float* __restrict__ part_o, float* __restrict__ part_ml) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* q_s = smem;                       // [H][256 B]
-  uint8_t* kv_s = smem + H * 256;            // [DTILE][256 B]
+  uint8_t* q_s = smem;                               // [H][256 B]
+  uint8_t* kv_s = smem + H * 256;                    // [SPLIT][256 B] dequantised entries
+  uint8_t* st_nope = kv_s + SPLIT * 256;             // [SPLIT][64 B]  FP8 codes as stored
+  uint8_t* st_rope = st_nope + SPLIT * kNope;        // [SPLIT][128 B] RoPE dims as stored
+  float* st_scale = reinterpret_cast<float*>(st_rope + SPLIT * kRope * 2);   // [SPLIT]
   __shared__ int32_t ent[SPLIT];
   const int b = blockIdx.y, sp = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -393,37 +396,53 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
     for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 
+  // the split's entries as stored (FP8 codes, RoPE dims, scale), all copies in
+  // flight at once; empty slots read as zeros
+  constexpr int PIECES = kNope / 16 + (kRope * 2) / 16 + 1;   // 16-byte pieces + the scale
+  for (int x = tid; x < SPLIT * PIECES; x += nthreads) {
+    const int row = x / PIECES, c = x - row * PIECES;
+    const int e = ent[row];
+    const size_t er = (size_t)b * n_max + (e < 0 ? 0 : e);
+    if (c < kNope / 16)
+      cp_async16(smem_u32(st_nope + row * kNope + c * 16), nope + er * kNope + c * 16, e >= 0);
+    else if (c < PIECES - 1)
+      cp_async16(smem_u32(st_rope + row * (kRope * 2) + (c - kNope / 16) * 16),
+                 reinterpret_cast<const uint8_t*>(rope + er * kRope) + (c - kNope / 16) * 16, e >= 0);
+    else
+      cp_async4(smem_u32(st_scale + row), kv_scale + er, e >= 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  // dequantise into the MMA layout: chunks 0..7 = FP8 dims x scale, 8..15 = RoPE dims
+  for (int x = tid; x < SPLIT * 16; x += nthreads) {
+    const int chunk = x & 15, row = x >> 4;
+    uint4 v;
+    if (chunk < 8) {
+      const uint2 c8 = *reinterpret_cast<const uint2*>(st_nope + row * kNope + chunk * 8);
+      const float sc = st_scale[row];
+      const uint32_t cw[2] = {c8.x, c8.y};
+      uint32_t ow[4];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] & 0xffffu), __NV_E4M3);
+        const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] >> 16), __NV_E4M3);
+        const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+        const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+        ow[2 * k] = pack_bf16x2(f01.x * sc, f01.y * sc);
+        ow[2 * k + 1] = pack_bf16x2(f23.x * sc, f23.y * sc);
+      }
+      v = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    } else {
+      v = *reinterpret_cast<const uint4*>(st_rope + row * (kRope * 2) + (chunk - 8) * 16);
+    }
+    *reinterpret_cast<uint4*>(kv_s + swz(row, chunk, 256)) = v;
+  }
+  __syncthreads();
+
   for (int t0 = 0; t0 < SPLIT; t0 += DTILE) {
     if (s0 + t0 >= n_slots) break;
-    // dequantise 64 entries into shared memory: chunks 0..7 FP8 dims, 8..15 RoPE dims
-    for (int x = tid; x < DTILE * 16; x += nthreads) {
-      const int chunk = x & 15, row = x >> 4;
-      const int e = ent[t0 + row];
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (e >= 0) {
-        const size_t er = (size_t)b * n_max + e;
-        if (chunk < 8) {
-          const uint2 c8 = __ldg(reinterpret_cast<const uint2*>(nope + er * kNope) + chunk);
-          const float sc = __ldg(kv_scale + er);
-          const uint32_t cw[2] = {c8.x, c8.y};
-          uint32_t ow[4];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] & 0xffffu), __NV_E4M3);
-            const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] >> 16), __NV_E4M3);
-            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-            ow[2 * k] = pack_bf16x2(f01.x * sc, f01.y * sc);
-            ow[2 * k + 1] = pack_bf16x2(f23.x * sc, f23.y * sc);
-          }
-          v = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-        } else {
-          v = __ldg(reinterpret_cast<const uint4*>(rope + er * kRope) + (chunk - 8));
-        }
-      }
-      *reinterpret_cast<uint4*>(kv_s + swz(row, chunk, 256)) = v;
-    }
-    __syncthreads();
+    const uint8_t* kv_t = kv_s + t0 * 256;   // this tile's 64 entries
     float s[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -436,7 +455,7 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
         uint32_t b0, b1, b2, b3;
         const int row = np * 16 + (lane & 7) + ((lane >> 4) << 3);
         const int chunk = ks * 2 + ((lane >> 3) & 1);
-        ldsm_x4(smem_u32(kv_s + swz(row, chunk, 256)), b0, b1, b2, b3);
+        ldsm_x4(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
         mma_bf16_16816(s[2 * np], qf[ks], b0, b1);
         mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
       }
@@ -494,7 +513,7 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
         uint32_t b0, b1, b2, b3;
         const int row = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
         const int chunk = dp * 2 + (lane >> 4);
-        ldsm_x4_t(smem_u32(kv_s + swz(row, chunk, 256)), b0, b1, b2, b3);
+        ldsm_x4_t(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
         mma_bf16_16816(o[2 * dp], pa, b0, b1);
         mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
       }
@@ -530,16 +549,30 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   const int n = min(n_entries[b], n_max);
   const int used = sparse ? min(splits, (min(topk, n) + SPLIT - 1) / SPLIT) : min(splits, (n + SPLIT - 1) / SPLIT);
   const float* pm = part_ml + (size_t)b * splits * H * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < used; ++s) M = fmaxf(M, pm[((size_t)s * H + h) * 2]);
-  float num = 0.f, den = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < used; ++s) {
-      const float ms = pm[((size_t)s * H + h) * 2];
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      den = fmaf(f, pm[((size_t)s * H + h) * 2 + 1], den);
-      num = fmaf(f, part_o[(((size_t)b * splits + s) * H + h) * kD + d], num);
+  const float* po = part_o + ((size_t)b * splits * H + h) * kD + d;
+  // one pass with a running maximum; the loads of 8 splits are issued together
+  float M = -INFINITY, num = 0.f, den = 0.f;
+  for (int s0 = 0; s0 < used; s0 += 8) {
+    float ms[8], ls[8], os[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int sp = s0 + i;
+      ms[i] = sp < used ? pm[((size_t)sp * H + h) * 2] : -INFINITY;
+      ls[i] = sp < used ? pm[((size_t)sp * H + h) * 2 + 1] : 0.f;
+      os[i] = sp < used ? po[(size_t)sp * H * kD] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (ms[i] == -INFINITY) continue;
+      if (ms[i] > M) {
+        const float a = M == -INFINITY ? 0.f : exp2f(M - ms[i]);
+        num *= a;
+        den *= a;
+        M = ms[i];
+      }
+      const float f = exp2f(ms[i] - M);
+      den = fmaf(f, ls[i], den);
+      num = fmaf(f, os[i], num);
     }
   }
   const float r = den > 0.f ? num / den : 0.f;
@@ -618,12 +651,12 @@ static cslc_status run_topk_stages(const float* scores, const int32_t* n_entries
 static cslc_status run_attention(const cslc_decode_layer& l, int B, int H, const int32_t* idx,
                                  DecodeWs& w, cudaStream_t stream) {
   const int splits = layer_splits(l);
-  const size_t smem = (size_t)H * 256 + DTILE * 256;
+  const size_t smem = (size_t)H * 256 + SPLIT * (256 + kNope + kRope * 2 + 4);
   static int configured_for = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_for != dev) {
-    const int max_smem = 128 * 256 + DTILE * 256;
+    const int max_smem = 128 * 256 + SPLIT * (256 + kNope + kRope * 2 + 4);
     cudaFuncSetAttribute(decode_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     cudaFuncSetAttribute(decode_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     configured_for = dev;
