@@ -183,7 +183,9 @@ class CsaPrefill:
         self.out = torch.empty_like(self.x["q"])
         nb = C.indexer_topk_workspace_bytes(s.B, s.L, s.n_c, s.HI, s.topk)
         self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
-        self.rows_per_block = nb // (s.B * s.n_c * 4)
+        # the library's blocking rule: rows of <= 512 MiB of fp32 scores per block
+        # (a multiple of 64 rows), two blocks in flight
+        self.rows_per_block = max(64, ((512 << 20) // (s.n_c * 4)) // 64 * 64)
         self.launches = 2 + 2 * math.ceil(s.L / self.rows_per_block)
         self.pairs = csa_selected_pairs(s.L, s.m, s.n_c, s.topk)
         self.flops_attn = 4.0 * 128 * s.H * self.pairs            # QK^T + PV over selected pairs

@@ -65,7 +65,7 @@ static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 // auxiliary stream beside the indexer of the next, so neither launch's tail
 // leaves SMs idle.
 static int score_block_rows(int Nc) {
-  const long long budget = 256ll << 20;   // bytes of scores per block
+  const long long budget = 512ll << 20;   // bytes of scores per block
   long long rows = budget / ((long long)Nc * 4);
   rows = rows < 64 ? 64 : rows;
   rows = (rows / 64) * 64;

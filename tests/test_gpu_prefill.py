@@ -134,10 +134,11 @@ def test_indexer_topk_blocks_in_flight(C):
     streams (three blocks here, so a buffer is reused): the selection equals
     the one made from the full score tensor, which the oracle checks on
     sampled rows."""
-    B, L, HI, m, topk, Nc = 1, 3000, 4, 4, 512, 45056
+    B, L, HI, m, topk, Nc = 1, 6000, 4, 4, 512, 45056
     q_pos0 = m * Nc - L
-    block_bytes = C.indexer_topk_workspace_bytes(B, L, Nc, HI, topk) // 2
-    assert 0 < 2 * block_bytes < B * L * Nc * 4        # two buffers, each under half the rows
+    block_bytes = C.indexer_topk_workspace_bytes(B, L, Nc, HI, topk) // 2   # two buffers
+    rows_per_block = block_bytes // (B * Nc * 4)
+    assert 0 < rows_per_block and -(-L // rows_per_block) >= 3
     s = W.PrefillShape(B=B, L=L, H=16, m=m, HI=HI, topk=topk)
     x = W.prefill_inputs(s, wid=41, with_indexer=True)
     x["k_idx"] = W.randn_bf16((B, Nc, 64), W.seed_of(41, W.T_KIDX))
