@@ -478,8 +478,8 @@ def profile_case(name):
 # kernel source is the one that was measured.
 MEASURED_TRAFFIC = {
     "sparse": {"src": "sparse_attn_sm100.cu",
-               "sha256": "2101640d3670ed965063b862bfbaae2461b012a8f3dda0224ae2bfd2f24ec7a0",
-               "bytes_per_token": (172.144128e6 + 100.620032e6) / 8192},
+               "sha256": "802c5958659538450baf7587a94be6f27bcd2214b5c8ac30757c51daabebb8ce",
+               "bytes_per_token": (172.393472e6 + 101.704960e6) / 8192},
     "dense": {"src": "dense_attn_sm100.cu",
               "sha256": "ebe369f7ee47983d6c170cdce3599d7512ba0773663d881cf2c7ec2cc447afd7",
               "bytes_per_token": (1.074352e9 + 1.022927e9) / 65536},
