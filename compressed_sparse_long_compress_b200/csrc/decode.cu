@@ -167,22 +167,23 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_hist_kernel(const float* _
 
 // Finds bin T with count(bins > T) < k <= count(bins >= T). Block-wide, DEC_THREADS.
 __device__ void find_threshold_bin(const uint32_t* gh, int k, int* out_bin, int* out_above) {
-  __shared__ uint32_t part[DEC_THREADS];
-  const int tid = threadIdx.x;
+  __shared__ uint32_t wsum[DEC_THREADS / 32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // thread t owns bins 4095-16t .. 4080-16t
   uint32_t cnt[16], s = 0;
 #pragma unroll
   for (int j = 0; j < 16; ++j) { cnt[j] = gh[HIST_BINS - 1 - 16 * tid - j]; s += cnt[j]; }
-  part[tid] = s;
-  __syncthreads();
-  // inclusive scan over threads (Hillis-Steele in shared memory)
-  for (int o = 1; o < DEC_THREADS; o <<= 1) {
-    const uint32_t v = tid >= o ? part[tid - o] : 0u;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
+  // inclusive scan over threads: warp shuffles, then the warps' totals
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
-  const uint32_t incl = part[tid], excl = incl - s;
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) incl += wsum[w];
+  const uint32_t excl = incl - s;
   if (excl < (uint32_t)k && incl >= (uint32_t)k) {
     uint32_t above = excl;
     for (int j = 0; j < 16; ++j) {
@@ -211,10 +212,21 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
   const uint32_t T = (uint32_t)thr[0];
   const int c1 = min(n, c0 + DEC_CHUNK);
   const unsigned lt = (1u << lane) - 1u;
-  for (int base = c0; base < c1; base += DEC_THREADS) {
+  // this thread's scores of the chunk, all loads in flight before any is used
+  constexpr int PER_THREAD = DEC_CHUNK / DEC_THREADS;
+  float sv[PER_THREAD];
+#pragma unroll
+  for (int i = 0; i < PER_THREAD; ++i) {
+    const int e = c0 + i * DEC_THREADS + tid;
+    sv[i] = e < c1 ? scores[(size_t)b * n_max + e] : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < PER_THREAD; ++i) {
+    const int base = c0 + i * DEC_THREADS;
+    if (base >= c1) break;
     const int e = base + tid;
     const bool valid = e < c1;
-    const uint32_t key = valid ? float_key(scores[(size_t)b * n_max + e]) : 0u;
+    const uint32_t key = valid ? float_key(sv[i]) : 0u;
     const uint32_t bin = key >> HIST_SHIFT;
     const bool above = valid && bin > T, inbin = valid && bin == T;
     const unsigned ma = __ballot_sync(0xffffffffu, above);
@@ -260,18 +272,24 @@ __global__ void __launch_bounds__(FIN_THREADS) decode_finalize_kernel(
   if (tid == 0) fill = n_above;
   __syncthreads();
 
-  // radix select of the need-th largest composite key among the C candidates
-  uint64_t prefix = 0, mask = 0;
+  // radix select of the need-th largest composite key among the C candidates;
+  // they all share the top HIST_BITS key bits (the threshold bin), so the
+  // digits start below those (8-bit digits, a last 4-bit one)
+  constexpr int FIXED = 64 - (32 - HIST_SHIFT);   // bits 63 .. FIXED are the bin
+  uint64_t prefix = C > 0 ? (cand_key(cb[0]) >> FIXED) << FIXED : 0ull;
+  uint64_t mask = ~0ull << FIXED;
   int remaining = need;
   bool take_all = (C == need);
-  for (int shift = 56; shift >= 0 && !take_all; shift -= 8) {
+  for (int shift = FIXED - 8; shift > -8 && !take_all; shift -= 8) {
+    const int sh = shift < 0 ? 0 : shift;                  // the last digit is narrower
+    const uint32_t dmask = shift < 0 ? (0xffu >> -shift) : 0xffu;
     for (int x = tid; x < (FIN_THREADS / 32) * 256; x += FIN_THREADS) (&hist[0][0])[x] = 0;
     if (tid == 0) { bc[0] = 0; bc[1] = 0; bc[2] = 0; }
     __syncthreads();
     for (int i = tid; i < C; i += FIN_THREADS) {
       const uint64_t k = cand_key(cb[i]);
       if ((k & mask) == prefix) {
-        const uint32_t d = (uint32_t)(k >> shift) & 255u;
+        const uint32_t d = (uint32_t)(k >> sh) & dmask;
         const unsigned peers = __match_any_sync(__activemask(), d);
         if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp][d], (uint32_t)__popc(peers));
       }
@@ -310,8 +328,8 @@ __global__ void __launch_bounds__(FIN_THREADS) decode_finalize_kernel(
     const int above = bc[1], cnt_d = bc[2];
     __syncthreads();
     remaining -= above;
-    prefix |= d << shift;
-    mask |= 255ull << shift;
+    prefix |= d << sh;
+    mask |= (uint64_t)dmask << sh;
     if (cnt_d == remaining) take_all = true;
   }
   // composite keys are unique, so after the last digit exactly `remaining` match
