@@ -218,27 +218,27 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
         }
         if (!ok) break;
         tc_fence_after();
+        // the tile's 128 scores of this row: all four TMEM loads before one wait
+        uint32_t sr[DA_TILE / 32][32];
+#pragma unroll
+        for (int c0 = 0; c0 < DA_TILE / 32; ++c0) tmem_ld32(tmem + lane_off + sb * 128 + c0 * 32, sr[c0]);
+        tmem_wait_ld();
         float s[DA_TILE];
 #pragma unroll
-        for (int c0 = 0; c0 < DA_TILE; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + sb * 128 + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[c0 + k] = __uint_as_float(r[k]);
-        }
+        for (int c = 0; c < DA_TILE; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
         const int lim = nv - j * DA_TILE;                   // entries of this tile the row sees
-        float mx = -INFINITY;
-        if (lim >= DA_TILE) {
+        if (lim < DA_TILE) {
 #pragma unroll
-          for (int c = 0; c < DA_TILE; ++c) mx = fmaxf(mx, s[c]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < DA_TILE; ++c) {
-            s[c] = c < lim ? s[c] : -INFINITY;
-            mx = fmaxf(mx, s[c]);
-          }
+          for (int c = 0; c < DA_TILE; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
+        // row maximum as 8 independent chains (max is exact in any order)
+        float mx8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx8[q] = s[q];
+#pragma unroll
+        for (int c = 8; c < DA_TILE; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         mx *= scale_log2;
         // lazy max: move it (and rescale O, l) only when it grows by more than 2^8
         const bool grow = mx > mrow + DA_GROW || (mrow == -INFINITY && mx != -INFINITY);
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
         // P = 2^(c*s - m): bf16, row-major (K-major A operand) in two 64-entry halves
         uint8_t* prow = p_s + pb * DA_TILE_BYTES;
         const float mneg = mrow == -INFINITY ? 0.f : -mrow;
-        float psum = 0.f;
+        float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent partial sums
 #pragma unroll
         for (int c8 = 0; c8 < 16; ++c8) {
           uint32_t pk[4];
@@ -280,13 +280,14 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
           for (int k = 0; k < 4; ++k) {
             const float a = ex2_approx(fmaf(s[8 * c8 + 2 * k], scale_log2, mneg));
             const float bq = ex2_approx(fmaf(s[8 * c8 + 2 * k + 1], scale_log2, mneg));
-            psum += a + bq;
+            ps8[2 * k] += a;
+            ps8[2 * k + 1] += bq;
             pk[k] = pack_bf16x2(a, bq);
           }
           *reinterpret_cast<uint4*>(prow + (c8 >> 3) * (DA_ROWS * 128) + sw128(row, c8 & 7)) =
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        lrow += psum;
+        lrow += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
