@@ -211,12 +211,11 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
       float mrow = -INFINITY, lrow = 0.f;
       for (int j = 0; j < nkv; ++j) {
         const int sb = s_it & 1, pb = p_it & 1;
-        {
-          bool w = true;
-          if (tid == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
-          ok = !named_bar_or(1, 128, !w);
-        }
-        if (!ok) break;
+        // each warp waits for S on its own; a failed wait is acted on at the
+        // tile's single vote below (reading TMEM is harmless meanwhile)
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&bars.s_full[sb], (uint32_t)((s_it >> 1) & 1), abortp, errp, ERR_S_FULL);
+        w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
         tc_fence_after();
         // the tile's 128 scores of this row: all four TMEM loads before one wait
         uint32_t sr[DA_TILE / 32][32];
@@ -249,11 +248,10 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
           lrow *= alpha;
         }
         const bool warp_rescale = __any_sync(0xffffffffu, grow && alpha != 0.f && j > 0);
-        if (warp_rescale) {
-          bool w = true;
+        if (warp_rescale && w) {
           if (lane == 0) w = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
-          ok = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
-          if (ok) {
+          w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+          if (w) {
             tc_fence_after();
 #pragma unroll
             for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -267,7 +265,7 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
             tmem_wait_st();
           }
         }
-        ok = !named_bar_or(1, 128, !ok);
+        ok = !named_bar_or(1, 128, !w || *abortp != 0);
         if (!ok) break;
         // P = 2^(c*s - m): bf16, row-major (K-major A operand) in two 64-entry halves
         uint8_t* prow = p_s + pb * DA_TILE_BYTES;
