@@ -481,8 +481,8 @@ MEASURED_TRAFFIC = {
                "sha256": "802c5958659538450baf7587a94be6f27bcd2214b5c8ac30757c51daabebb8ce",
                "bytes_per_token": (172.393472e6 + 101.704960e6) / 8192},
     "dense": {"src": "dense_attn_sm100.cu",
-              "sha256": "ebe369f7ee47983d6c170cdce3599d7512ba0773663d881cf2c7ec2cc447afd7",
-              "bytes_per_token": (1.074352e9 + 1.022927e9) / 65536},
+              "sha256": "af36d8a4718ffbb150d354dde250f6ce60a0ab0c0ef2dae763644e1b8e6a32e1",
+              "bytes_per_token": (1.074968e9 + 1.023328e9) / 65536},
 }
 
 
