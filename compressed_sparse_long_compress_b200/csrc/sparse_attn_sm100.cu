@@ -16,10 +16,10 @@
 //   warps 0-7   softmax + epilogue. Warp w owns TMEM lane quadrant w & 3 (32
 //               entries of the tile, or 32 output dims) and head half w >> 2,
 //               so two warps share each SM sub-partition. The per-head
-//               running max m[h] is CTA-wide and only moved (exact tile max
-//               by warp reduction, O^T rescale in TMEM) on a token's first
-//               tile or when a probability would exceed 2^8 -- rare after the
-//               first tile. P^T rows go to 128-byte-swizzled shared memory.
+//               reference m[h] is CTA-wide: on a token's first tile it is the
+//               score of the token's first valid entry, and it only moves
+//               (exact tile max by warp reduction, O^T rescale in TMEM) when a
+//               probability would exceed 2^8. P^T rows go to 128-byte-swizzled shared memory.
 //               At the token's end the head sums are reduced (butterfly
 //               reduce-scatter), O^T is read from TMEM, normalised,
 //               transposed through shared memory and stored.
@@ -80,6 +80,8 @@ struct SaSmall {
   int abort_flag;
   int n_tiles[2];
   int last_w[2][4];
+  int first_w[2][4];
+  int ref_slot[2];     // first valid slot of the token (the softmax reference row), or SA_MAXK
   int any_rescale;
   __align__(16) float mref[SA_NP];   // running max per head (log2 units of c*S)
   __align__(16) float alpha[SA_NP];
@@ -189,19 +191,27 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
       }
       const int32_t* irow = idx + g * (long long)topk;
       int32_t* is = idx_s + qb * SA_MAXK;
-      int last = 0;
+      int last = 0, first = SA_MAXK;
       for (int s = p; s < topk; s += SA_NPROD) {
         int e = __ldg(irow + s);
         if (e < 0 || e >= Nc) e = -1;
         is[s] = e;
-        if (e >= 0) last = s + 1;
+        if (e >= 0) {
+          last = s + 1;
+          first = min(first, s);
+        }
       }
       last = __reduce_max_sync(0xffffffffu, last);
-      if (lane == 0) sm->last_w[qb][p >> 5] = last;
+      first = __reduce_min_sync(0xffffffffu, first);
+      if (lane == 0) {
+        sm->last_w[qb][p >> 5] = last;
+        sm->first_w[qb][p >> 5] = first;
+      }
       named_bar(1, SA_NPROD);
       const int nt = (max(max(sm->last_w[qb][0], sm->last_w[qb][1]), sm->last_w[qb][2]) + SA_TILE - 1) / SA_TILE;
       if (p == 0) {
         sm->n_tiles[qb] = nt;
+        sm->ref_slot[qb] = min(min(sm->first_w[qb][0], sm->first_w[qb][1]), sm->first_w[qb][2]);
         uint8_t* qd = q_s + qb * SA_Q_BYTES;
         mbar_arrive_expect_tx(&bars.tok_full[qb], (uint32_t)(H * 256));
         tma_load_2d(qd, &tm_q, 0, (int)(g * H), &bars.tok_full[qb]);
@@ -277,29 +287,59 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
         const int slot = j * SA_TILE + row;
         const bool valid = slot < topk && is[slot] >= 0;
-        float v[HT];
-        float pmax = 0.f;
-        if (w) {
-          tc_fence_after();
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + sb * 64 + h0, r);
-          tmem_wait_ld();
-          if (valid && j > 0) {
+        // On a token's first tile the reference m[h] is the score of the
+        // token's first valid entry (its probability is exactly 1, so nothing
+        // underflows); a tile whose probabilities would exceed 2^8 against it
+        // takes the exact-max path below. Without a valid entry in the first
+        // tile the exact-max path runs directly.
+        bool ref_ok = true;
+        if (j == 0) {
+          const int rs = sm->ref_slot[qb];
+          ref_ok = rs < SA_TILE;
+          if (w && ref_ok && q4 == (rs >> 5)) {   // the warps holding that row (warp-uniform)
+            tc_fence_after();
+            uint32_t rr[32];
+            tmem_ld32(tmem + lane_off + sb * 64 + h0, rr);
+            tmem_wait_ld();
+            if (row == rs) {
 #pragma unroll
-            for (int h = 0; h < HT; ++h) {
-              v[h] = ex2_approx(fmaf(__uint_as_float(r[h]), scale_log2, negm[h]));
-              pmax = fmaxf(pmax, v[h]);
+              for (int h4 = 0; h4 < HT; h4 += 4)
+                *reinterpret_cast<float4*>(&sm->mref[h0 + h4]) =
+                    make_float4(__uint_as_float(rr[h4]) * scale_log2, __uint_as_float(rr[h4 + 1]) * scale_log2,
+                                __uint_as_float(rr[h4 + 2]) * scale_log2, __uint_as_float(rr[h4 + 3]) * scale_log2);
             }
-          } else {
+          }
+          named_bar(2, SA_NSOFT);
+          if (ref_ok) {
 #pragma unroll
-            for (int h = 0; h < HT; ++h) v[h] = 0.f;
+            for (int h4 = 0; h4 < HT; h4 += 4) {
+              const float4 m4 = *reinterpret_cast<const float4*>(&sm->mref[h0 + h4]);
+              negm[h4] = -m4.x; negm[h4 + 1] = -m4.y; negm[h4 + 2] = -m4.z; negm[h4 + 3] = -m4.w;
+            }
           }
         }
-        // j == 0 always takes the exact-max path (negm starts at +inf). A raised
-        // abort flag joins the vote, so that all softmax warps leave together
-        // (the named barriers stay matched).
+        uint32_t r[32];
+        if (w) {
+          tc_fence_after();
+          tmem_ld32(tmem + lane_off + sb * 64 + h0, r);
+          tmem_wait_ld();
+        }
+        float v[HT];
+        float pmax = 0.f;
+        if (w && valid && ref_ok) {
+#pragma unroll
+          for (int h = 0; h < HT; ++h) {
+            v[h] = ex2_approx(fmaf(__uint_as_float(r[h]), scale_log2, negm[h]));
+            pmax = fmaxf(pmax, v[h]);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < HT; ++h) v[h] = 0.f;
+        }
+        // A raised abort flag joins the vote, so that all softmax warps leave
+        // together (the named barriers stay matched).
         bool slow = false;
-        if (named_bar_or(3, SA_NSOFT, j == 0 || !(pmax <= SA_OVERFLOW) || !w || *abortp != 0)) {
+        if (named_bar_or(3, SA_NSOFT, !ref_ok || !(pmax <= SA_OVERFLOW) || !w || *abortp != 0)) {
           if (named_bar_or(3, SA_NSOFT, !w || *abortp != 0)) { ok = false; break; }
           slow = true;
         }
