@@ -12,15 +12,24 @@
 //                          histogram of the score keys (top 12 bits)
 //   decode_select_kernel   finds the histogram bin holding the k-th largest
 //                          score; entries above it are selected, entries in it
-//                          become candidates
+//                          become candidates (a block scan places them; one
+//                          atomic per counter and CTA)
 //   decode_finalize_kernel exact choice among the candidates (64-bit radix
 //                          select on score key ++ reversed index, so ties go to
-//                          the smaller index), then a bitonic sort of the k
-//                          indices into ascending order
-//   decode_attn_kernel     split-K attention: each CTA dequantises 128 entries
-//                          (e4m3 * scale -> bf16, RoPE half copied) into shared
-//                          memory and runs QK^T / softmax / PV for all heads
+//                          the smaller index), then the k indices in ascending
+//                          order through a bitmap of the context and a block
+//                          scan (a bitonic sort above 262,144 entries)
+//   decode_attn_kernel     split-K attention: each CTA takes one or more chunks
+//                          of 128 entries (about two CTAs per SM over the
+//                          layer); a chunk's stored entries are staged with
+//                          one batch of cp.async while the previous chunk is
+//                          computed, dequantised (e4m3 * scale -> bf16, RoPE
+//                          half copied) into shared memory, and QK^T / softmax
+//                          / PV run for all heads
 //   decode_combine_kernel  merges the splits with their max / sum statistics
+//                          (two thread groups, each over half of the splits)
+
+#include <algorithm>
 
 #include "common.cuh"
 
@@ -30,7 +39,8 @@ constexpr int DEC_CHUNK = 4096;      // entries per scores / select CTA
 constexpr int DEC_THREADS = 256;
 constexpr int HIST_BINS = 4096;      // top 12 bits of the score key
 constexpr int HIST_SHIFT = 20;
-constexpr int SPLIT = 128;           // entries per attention CTA
+constexpr int SPLIT = 128;           // entries per attention chunk (a CTA takes one or more)
+constexpr int ATTN_CTAS = 296;       // attention CTAs aimed at per layer: two per SM on 148 SMs
 constexpr int DTILE = 64;            // entries per attention tile
 constexpr int FIN_THREADS = 1024;
 constexpr int MAX_TOPK = 2048;
@@ -211,36 +221,62 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
   find_threshold_bin(ghist + (size_t)b * HIST_BINS, topk, &thr[0], &thr[1]);
   const uint32_t T = (uint32_t)thr[0];
   const int c1 = min(n, c0 + DEC_CHUNK);
-  const unsigned lt = (1u << lane) - 1u;
   // this thread's scores of the chunk, all loads in flight before any is used
   constexpr int PER_THREAD = DEC_CHUNK / DEC_THREADS;
+  static_assert(PER_THREAD <= 16, "per-thread flags fit 16 bits");
   float sv[PER_THREAD];
 #pragma unroll
   for (int i = 0; i < PER_THREAD; ++i) {
     const int e = c0 + i * DEC_THREADS + tid;
     sv[i] = e < c1 ? scores[(size_t)b * n_max + e] : 0.f;
   }
+  uint32_t fa = 0u, fc = 0u;   // bit i: score i is above / inside the threshold bin
 #pragma unroll
   for (int i = 0; i < PER_THREAD; ++i) {
-    const int base = c0 + i * DEC_THREADS;
-    if (base >= c1) break;
-    const int e = base + tid;
-    const bool valid = e < c1;
-    const uint32_t key = valid ? float_key(sv[i]) : 0u;
-    const uint32_t bin = key >> HIST_SHIFT;
-    const bool above = valid && bin > T, inbin = valid && bin == T;
-    const unsigned ma = __ballot_sync(0xffffffffu, above);
-    const unsigned mc = __ballot_sync(0xffffffffu, inbin);
-    int base_a = 0, base_c = 0;
-    if (lane == 0) {
-      if (ma) base_a = atomicAdd(&counters[2 * b], __popc(ma));
-      if (mc) base_c = atomicAdd(&counters[2 * b + 1], __popc(mc));
+    const int e = c0 + i * DEC_THREADS + tid;
+    const uint32_t bin = float_key(sv[i]) >> HIST_SHIFT;
+    if (e < c1 && bin > T) fa |= 1u << i;
+    if (e < c1 && bin == T) fc |= 1u << i;
+  }
+  // block exclusive scan of (above count << 16 | candidate count); one atomic
+  // per counter and CTA reserves the CTA's output ranges
+  __shared__ uint32_t wtot[DEC_THREADS / 32];
+  __shared__ int base[2];
+  const int warp = tid >> 5;
+  const uint32_t mine = ((uint32_t)__popc(fa) << 16) | (uint32_t)__popc(fc);
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0u, total = 0u;
+#pragma unroll
+  for (int w = 0; w < DEC_THREADS / 32; ++w) {
+    const uint32_t t = wtot[w];
+    if (w < warp) before += t;
+    total += t;
+  }
+  if (tid == 0) {
+    base[0] = (total >> 16) ? atomicAdd(&counters[2 * b], (int)(total >> 16)) : 0;
+    base[1] = (total & 0xffffu) ? atomicAdd(&counters[2 * b + 1], (int)(total & 0xffffu)) : 0;
+  }
+  __syncthreads();
+  const uint32_t excl = before + incl - mine;
+  int pa = base[0] + (int)(excl >> 16), pc = base[1] + (int)(excl & 0xffffu);
+#pragma unroll
+  for (int i = 0; i < PER_THREAD; ++i) {
+    const int e = c0 + i * DEC_THREADS + tid;
+    if ((fa >> i) & 1u) {
+      if (pa < MAX_TOPK) sel[(size_t)b * MAX_TOPK + pa] = e;
+      ++pa;
     }
-    base_a = __shfl_sync(0xffffffffu, base_a, 0);
-    base_c = __shfl_sync(0xffffffffu, base_c, 0);
-    const int pa = base_a + __popc(ma & lt), pc = base_c + __popc(mc & lt);
-    if (above && pa < MAX_TOPK) sel[(size_t)b * MAX_TOPK + pa] = e;
-    if (inbin && pc < n_max) cand[(size_t)b * n_max + pc] = make_uint2(key, (uint32_t)e);
+    if ((fc >> i) & 1u) {
+      if (pc < n_max) cand[(size_t)b * n_max + pc] = make_uint2(float_key(sv[i]), (uint32_t)e);
+      ++pc;
+    }
   }
 }
 
@@ -343,7 +379,57 @@ __global__ void __launch_bounds__(FIN_THREADS) decode_finalize_kernel(
     }
   }
   __syncthreads();
-  // bitonic sort of list[0..topk) ascending, padded to a power of two
+  if (n <= FIN_THREADS * 8 * 32) {
+    // ascending order through a bitmap of the context (the radix histogram's
+    // 8192 words): each thread owns 8 words, a block scan of their bit counts
+    // gives every thread its first output position
+    uint32_t* bm = &hist[0][0];
+    for (int x = tid; x < FIN_THREADS * 8; x += FIN_THREADS) bm[x] = 0u;
+    __syncthreads();
+    const int n_sel = min(fill, topk);
+    for (int j = tid; j < n_sel; j += FIN_THREADS) atomicOr(&bm[list[j] >> 5], 1u << (list[j] & 31));
+    __syncthreads();
+    uint32_t wv[8];
+    int cnt = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      wv[k] = bm[tid * 8 + k];
+      cnt += __popc(wv[k]);
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    __shared__ int wsum[FIN_THREADS / 32];
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int t = wsum[lane];
+      int ti = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, ti, o);
+        if (lane >= o) ti += v;
+      }
+      wsum[lane] = ti - t;   // exclusive prefix of the warp totals
+    }
+    __syncthreads();
+    int pos = wsum[warp] + incl - cnt;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t w = wv[k];
+      while (w) {
+        const int bit = __ffs(w) - 1;
+        out[pos++] = (tid * 8 + k) * 32 + bit;
+        w &= w - 1;
+      }
+    }
+    for (int j = n_sel + tid; j < topk; j += FIN_THREADS) out[j] = -1;
+    return;
+  }
+  // larger contexts: bitonic sort of list[0..topk) ascending, padded to a power of two
   int P = 1;
   while (P < topk) P <<= 1;
   for (int j = topk + tid; j < P; j += FIN_THREADS) list[j] = 0x7fffffff;
@@ -370,36 +456,64 @@ template <bool SPARSE>
 __global__ void __launch_bounds__(256) decode_attn_kernel(
     const uint16_t* __restrict__ q, const uint8_t* __restrict__ nope, const uint16_t* __restrict__ rope,
     const float* __restrict__ kv_scale, const int32_t* __restrict__ n_entries, int n_max,
-    const int32_t* __restrict__ idx, int topk, int H, float scale_log2, int splits,
+    const int32_t* __restrict__ idx, int topk, int H, float scale_log2, int splits, int chunks,
     float* __restrict__ part_o, float* __restrict__ part_ml) {
+  constexpr int ST_BYTES = SPLIT * (kNope + kRope * 2 + 4);   // one chunk as stored
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* q_s = smem;                               // [H][256 B]
   uint8_t* kv_s = smem + H * 256;                    // [SPLIT][256 B] dequantised entries
-  uint8_t* st_nope = kv_s + SPLIT * 256;             // [SPLIT][64 B]  FP8 codes as stored
-  uint8_t* st_rope = st_nope + SPLIT * kNope;        // [SPLIT][128 B] RoPE dims as stored
-  float* st_scale = reinterpret_cast<float*>(st_rope + SPLIT * kRope * 2);   // [SPLIT]
-  __shared__ int32_t ent[SPLIT];
+  uint8_t* st_base = kv_s + SPLIT * 256;             // [2] x (FP8 codes [SPLIT][64 B], RoPE dims
+                                                     //        [SPLIT][128 B], scales [SPLIT])
+  __shared__ int32_t ent_buf[2][SPLIT];
   const int b = blockIdx.y, sp = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nthreads = (H / 16) * 32;
   const int g = lane >> 2, tq = lane & 3;
   const int n = min(n_entries[b], n_max);
-  const int s0 = sp * SPLIT;
   const int n_slots = SPARSE ? topk : n;
+  const int slot0 = sp * chunks * SPLIT;
+  // chunks of this CTA that hold a slot (the rest of the split is past the end)
+  const int n_chunks = slot0 >= n_slots ? 0 : min(chunks, (n_slots - slot0 + SPLIT - 1) / SPLIT);
 
   for (int x = tid; x < H * 16; x += nthreads) {
     const int chunk = x & 15, row = x >> 4;
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)b * H + row) * kD) + chunk);
     *reinterpret_cast<uint4*>(q_s + swz(row, chunk, 256)) = v;
   }
-  for (int j = tid; j < SPLIT; j += nthreads) {
-    const int slot = s0 + j;
-    int e = -1;
-    if (slot < n_slots) e = SPARSE ? idx[(size_t)b * topk + slot] : slot;
-    if (e >= n) e = -1;
-    ent[j] = e;
-  }
+  // the entries of chunk c (-1 for empty slots) into ent_buf[c & 1]
+  auto fill_ent = [&](int c) {
+    for (int j = tid; j < SPLIT; j += nthreads) {
+      const int slot = slot0 + c * SPLIT + j;
+      int e = -1;
+      if (slot < n_slots) e = SPARSE ? idx[(size_t)b * topk + slot] : slot;
+      if (e >= n) e = -1;
+      ent_buf[c & 1][j] = e;
+    }
+  };
+  // the stored entries of chunk c, all copies in flight at once; empty slots read as zeros
+  constexpr int PIECES = kNope / 16 + (kRope * 2) / 16 + 1;   // 16-byte pieces + the scale
+  auto stage_chunk = [&](int c) {
+    uint8_t* st_nope = st_base + (c & 1) * ST_BYTES;
+    uint8_t* st_rope = st_nope + SPLIT * kNope;
+    float* st_scale = reinterpret_cast<float*>(st_rope + SPLIT * kRope * 2);
+    const int32_t* ent = ent_buf[c & 1];
+    for (int x = tid; x < SPLIT * PIECES; x += nthreads) {
+      const int row = x / PIECES, pc = x - row * PIECES;
+      const int e = ent[row];
+      const size_t er = (size_t)b * n_max + (e < 0 ? 0 : e);
+      if (pc < kNope / 16)
+        cp_async16(smem_u32(st_nope + row * kNope + pc * 16), nope + er * kNope + pc * 16, e >= 0);
+      else if (pc < PIECES - 1)
+        cp_async16(smem_u32(st_rope + row * (kRope * 2) + (pc - kNope / 16) * 16),
+                   reinterpret_cast<const uint8_t*>(rope + er * kRope) + (pc - kNope / 16) * 16, e >= 0);
+      else
+        cp_async4(smem_u32(st_scale + row), kv_scale + er, e >= 0);
+    }
+    cp_async_commit();
+  };
+  if (n_chunks > 0) fill_ent(0);
   __syncthreads();
+  if (n_chunks > 0) stage_chunk(0);
   uint32_t qf[8][4];
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
@@ -414,129 +528,130 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
     for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 
-  // the split's entries as stored (FP8 codes, RoPE dims, scale), all copies in
-  // flight at once; empty slots read as zeros
-  constexpr int PIECES = kNope / 16 + (kRope * 2) / 16 + 1;   // 16-byte pieces + the scale
-  for (int x = tid; x < SPLIT * PIECES; x += nthreads) {
-    const int row = x / PIECES, c = x - row * PIECES;
-    const int e = ent[row];
-    const size_t er = (size_t)b * n_max + (e < 0 ? 0 : e);
-    if (c < kNope / 16)
-      cp_async16(smem_u32(st_nope + row * kNope + c * 16), nope + er * kNope + c * 16, e >= 0);
-    else if (c < PIECES - 1)
-      cp_async16(smem_u32(st_rope + row * (kRope * 2) + (c - kNope / 16) * 16),
-                 reinterpret_cast<const uint8_t*>(rope + er * kRope) + (c - kNope / 16) * 16, e >= 0);
-    else
-      cp_async4(smem_u32(st_scale + row), kv_scale + er, e >= 0);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  // dequantise into the MMA layout: chunks 0..7 = FP8 dims x scale, 8..15 = RoPE dims
-  for (int x = tid; x < SPLIT * 16; x += nthreads) {
-    const int chunk = x & 15, row = x >> 4;
-    uint4 v;
-    if (chunk < 8) {
-      const uint2 c8 = *reinterpret_cast<const uint2*>(st_nope + row * kNope + chunk * 8);
-      const float sc = st_scale[row];
-      const uint32_t cw[2] = {c8.x, c8.y};
-      uint32_t ow[4];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] & 0xffffu), __NV_E4M3);
-        const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] >> 16), __NV_E4M3);
-        const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-        const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-        ow[2 * k] = pack_bf16x2(f01.x * sc, f01.y * sc);
-        ow[2 * k + 1] = pack_bf16x2(f23.x * sc, f23.y * sc);
-      }
-      v = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  for (int c = 0; c < n_chunks; ++c) {
+    // the next chunk's copies go out before this chunk is waited for
+    if (c + 1 < n_chunks) {
+      fill_ent(c + 1);
+      __syncthreads();
+      stage_chunk(c + 1);
+      cp_async_wait<1>();
     } else {
-      v = *reinterpret_cast<const uint4*>(st_rope + row * (kRope * 2) + (chunk - 8) * 16);
+      cp_async_wait<0>();
     }
-    *reinterpret_cast<uint4*>(kv_s + swz(row, chunk, 256)) = v;
-  }
-  __syncthreads();
-
-  for (int t0 = 0; t0 < SPLIT; t0 += DTILE) {
-    if (s0 + t0 >= n_slots) break;
-    const uint8_t* kv_t = kv_s + t0 * 256;   // this tile's 64 entries
-    float s[8][4];
+    __syncthreads();
+    const int32_t* ent = ent_buf[c & 1];
+    const int s0 = slot0 + c * SPLIT;
+    {
+      // dequantise into the MMA layout: chunks 0..7 = FP8 dims x scale, 8..15 = RoPE dims
+      const uint8_t* st_nope = st_base + (c & 1) * ST_BYTES;
+      const uint8_t* st_rope = st_nope + SPLIT * kNope;
+      const float* st_scale = reinterpret_cast<const float*>(st_rope + SPLIT * kRope * 2);
+      for (int x = tid; x < SPLIT * 16; x += nthreads) {
+        const int chunk = x & 15, row = x >> 4;
+        uint4 v;
+        if (chunk < 8) {
+          const uint2 c8 = *reinterpret_cast<const uint2*>(st_nope + row * kNope + chunk * 8);
+          const float sc = st_scale[row];
+          const uint32_t cw[2] = {c8.x, c8.y};
+          uint32_t ow[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) s[i][j] = 0.f;
-#pragma unroll
-    for (int np = 0; np < 4; ++np) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t b0, b1, b2, b3;
-        const int row = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int chunk = ks * 2 + ((lane >> 3) & 1);
-        ldsm_x4(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
-        mma_bf16_16816(s[2 * np], qf[ks], b0, b1);
-        mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
-      }
-    }
-    float tmax[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const bool valid = ent[t0 + nt * 8 + 2 * tq + j] >= 0;
-        const float v0 = valid ? s[nt][j] * scale_log2 : -INFINITY;
-        const float v1 = valid ? s[nt][2 + j] * scale_log2 : -INFINITY;
-        s[nt][j] = v0;
-        s[nt][2 + j] = v1;
-        tmax[0] = fmaxf(tmax[0], v0);
-        tmax[1] = fmaxf(tmax[1], v1);
-      }
-    }
-    float alpha[2], mnew[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
-      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
-      mnew[r] = fmaxf(mrow[r], tmax[r]);
-      alpha[r] = mrow[r] == -INFINITY ? 0.f : exp2f(mrow[r] - mnew[r]);
-      mrow[r] = mnew[r];
-    }
-    float psum[2] = {0.f, 0.f};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = j >> 1;
-        const float p = mnew[r] == -INFINITY ? 0.f : exp2f(s[nt][j] - mnew[r]);
-        s[nt][j] = p;
-        psum[r] += p;
-      }
-    }
-    lrow[0] = lrow[0] * alpha[0] + psum[0];
-    lrow[1] = lrow[1] * alpha[1] + psum[1];
-#pragma unroll
-    for (int dn = 0; dn < 16; ++dn) {
-      o[dn][0] *= alpha[0]; o[dn][1] *= alpha[0];
-      o[dn][2] *= alpha[1]; o[dn][3] *= alpha[1];
-    }
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
-      pa[1] = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
-      pa[2] = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-      pa[3] = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
-#pragma unroll
-      for (int dp = 0; dp < 8; ++dp) {
-        uint32_t b0, b1, b2, b3;
-        const int row = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int chunk = dp * 2 + (lane >> 4);
-        ldsm_x4_t(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * dp], pa, b0, b1);
-        mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+          for (int k = 0; k < 2; ++k) {
+            const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] & 0xffffu), __NV_E4M3);
+            const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] >> 16), __NV_E4M3);
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+            ow[2 * k] = pack_bf16x2(f01.x * sc, f01.y * sc);
+            ow[2 * k + 1] = pack_bf16x2(f23.x * sc, f23.y * sc);
+          }
+          v = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        } else {
+          v = *reinterpret_cast<const uint4*>(st_rope + row * (kRope * 2) + (chunk - 8) * 16);
+        }
+        *reinterpret_cast<uint4*>(kv_s + swz(row, chunk, 256)) = v;
       }
     }
     __syncthreads();
+
+    for (int t0 = 0; t0 < SPLIT; t0 += DTILE) {
+      if (s0 + t0 >= n_slots) break;
+      const uint8_t* kv_t = kv_s + t0 * 256;   // this tile's 64 entries
+      float s[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[i][j] = 0.f;
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          const int row = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int chunk = ks * 2 + ((lane >> 3) & 1);
+          ldsm_x4(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
+          mma_bf16_16816(s[2 * np], qf[ks], b0, b1);
+          mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
+        }
+      }
+      float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const bool valid = ent[t0 + nt * 8 + 2 * tq + j] >= 0;
+          const float v0 = valid ? s[nt][j] * scale_log2 : -INFINITY;
+          const float v1 = valid ? s[nt][2 + j] * scale_log2 : -INFINITY;
+          s[nt][j] = v0;
+          s[nt][2 + j] = v1;
+          tmax[0] = fmaxf(tmax[0], v0);
+          tmax[1] = fmaxf(tmax[1], v1);
+        }
+      }
+      float alpha[2], mnew[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
+        tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
+        mnew[r] = fmaxf(mrow[r], tmax[r]);
+        alpha[r] = mrow[r] == -INFINITY ? 0.f : exp2f(mrow[r] - mnew[r]);
+        mrow[r] = mnew[r];
+      }
+      float psum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = j >> 1;
+          const float p = mnew[r] == -INFINITY ? 0.f : exp2f(s[nt][j] - mnew[r]);
+          s[nt][j] = p;
+          psum[r] += p;
+        }
+      }
+      lrow[0] = lrow[0] * alpha[0] + psum[0];
+      lrow[1] = lrow[1] * alpha[1] + psum[1];
+#pragma unroll
+      for (int dn = 0; dn < 16; ++dn) {
+        o[dn][0] *= alpha[0]; o[dn][1] *= alpha[0];
+        o[dn][2] *= alpha[1]; o[dn][3] *= alpha[1];
+      }
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
+        pa[1] = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
+        pa[2] = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+        pa[3] = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+        for (int dp = 0; dp < 8; ++dp) {
+          uint32_t b0, b1, b2, b3;
+          const int row = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+          const int chunk = dp * 2 + (lane >> 4);
+          ldsm_x4_t(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
+          mma_bf16_16816(o[2 * dp], pa, b0, b1);
+          mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+        }
+      }
+      __syncthreads();
+    }
   }
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -558,23 +673,27 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
   }
 }
 
-__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
-                                                             const float* __restrict__ part_ml,
-                                                             const int32_t* __restrict__ n_entries,
-                                                             int n_max, int topk, int sparse, int H,
-                                                             int splits, uint16_t* __restrict__ out) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(2 * kD) decode_combine_kernel(const float* __restrict__ part_o,
+                                                                const float* __restrict__ part_ml,
+                                                                const int32_t* __restrict__ n_entries,
+                                                                int n_max, int topk, int sparse, int H,
+                                                                int splits, int split_slots,
+                                                                uint16_t* __restrict__ out) {
+  __shared__ float xm[kD], xn[kD], xd[kD];
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x & (kD - 1), grp = threadIdx.x / kD;
   const int n = min(n_entries[b], n_max);
-  const int used = sparse ? min(splits, (min(topk, n) + SPLIT - 1) / SPLIT) : min(splits, (n + SPLIT - 1) / SPLIT);
+  const int slots = sparse ? min(topk, n) : n;
+  const int used = min(splits, (slots + split_slots - 1) / split_slots);
   const float* pm = part_ml + (size_t)b * splits * H * 2;
   const float* po = part_o + ((size_t)b * splits * H + h) * kD + d;
-  // one pass with a running maximum; the loads of 8 splits are issued together
+  // each group takes every other split, one pass with a running maximum; the
+  // loads of 8 splits are issued together
   float M = -INFINITY, num = 0.f, den = 0.f;
-  for (int s0 = 0; s0 < used; s0 += 8) {
+  for (int s0 = 0; s0 < used; s0 += 16) {
     float ms[8], ls[8], os[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int sp = s0 + i;
+      const int sp = s0 + 2 * i + grp;
       ms[i] = sp < used ? pm[((size_t)sp * H + h) * 2] : -INFINITY;
       ls[i] = sp < used ? pm[((size_t)sp * H + h) * 2 + 1] : 0.f;
       os[i] = sp < used ? po[(size_t)sp * H * kD] : 0.f;
@@ -593,8 +712,23 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
       num = fmaf(f, os[i], num);
     }
   }
-  const float r = den > 0.f ? num / den : 0.f;
-  out[((size_t)b * H + h) * kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+  if (grp == 1) {
+    xm[d] = M;
+    xn[d] = num;
+    xd[d] = den;
+  }
+  __syncthreads();
+  if (grp == 0) {
+    const float Mo = xm[d];
+    if (Mo != -INFINITY) {
+      const float Mn = fmaxf(M, Mo);
+      const float a = M == -INFINITY ? 0.f : exp2f(M - Mn), c = exp2f(Mo - Mn);
+      num = num * a + xn[d] * c;
+      den = den * a + xd[d] * c;
+    }
+    const float r = den > 0.f ? num / den : 0.f;
+    out[((size_t)b * H + h) * kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+  }
 }
 
 // -------------------------------------------------------------- host side
@@ -606,9 +740,16 @@ struct DecodeWsSizes {
   size_t total() const { return scores + hist + counters + sel + cand + idx + part_o + part_ml; }
 };
 
-static int layer_splits(const cslc_decode_layer& l) {
+// chunks of SPLIT entries per attention CTA: about ATTN_CTAS CTAs over the layer
+static int layer_chunks(const cslc_decode_layer& l, int B) {
   const int slots = l.kind == 0 ? l.topk : l.n_max;
-  return slots > 0 ? (slots + SPLIT - 1) / SPLIT : 1;
+  const long long total = slots > 0 ? (long long)B * ((slots + SPLIT - 1) / SPLIT) : 0;
+  return (int)std::max<long long>(1, (total + ATTN_CTAS - 1) / ATTN_CTAS);
+}
+static int layer_splits(const cslc_decode_layer& l, int B) {
+  const int slots = l.kind == 0 ? l.topk : l.n_max;
+  const int per = SPLIT * layer_chunks(l, B);
+  return slots > 0 ? (slots + per - 1) / per : 1;
 }
 
 static DecodeWsSizes ws_sizes(int B, int n_max, int topk, int splits, int H) {
@@ -628,7 +769,7 @@ size_t decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers, int
   size_t best = 0;
   for (int i = 0; i < n_layers; ++i) {
     const cslc_decode_layer& l = layers[i];
-    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l), H);
+    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l, B), H);
     if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
     best = s.total() > best ? s.total() : best;
   }
@@ -668,13 +809,13 @@ static cslc_status run_topk_stages(const float* scores, const int32_t* n_entries
 
 static cslc_status run_attention(const cslc_decode_layer& l, int B, int H, const int32_t* idx,
                                  DecodeWs& w, cudaStream_t stream) {
-  const int splits = layer_splits(l);
-  const size_t smem = (size_t)H * 256 + SPLIT * (256 + kNope + kRope * 2 + 4);
+  const int chunks = layer_chunks(l, B), splits = layer_splits(l, B);
+  const size_t smem = (size_t)H * 256 + SPLIT * 256 + 2 * SPLIT * (kNope + kRope * 2 + 4);
   static int configured_for = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_for != dev) {
-    const int max_smem = 128 * 256 + SPLIT * (256 + kNope + kRope * 2 + 4);
+    const int max_smem = 128 * 256 + SPLIT * 256 + 2 * SPLIT * (kNope + kRope * 2 + 4);
     cudaFuncSetAttribute(decode_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     cudaFuncSetAttribute(decode_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     configured_for = dev;
@@ -683,14 +824,16 @@ static cslc_status run_attention(const cslc_decode_layer& l, int B, int H, const
   const float sl2 = l.scale * kLog2e;
   if (l.kind == 0)
     decode_attn_kernel<true><<<grid, (H / 16) * 32, smem, stream>>>(
-        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, idx, l.topk, H, sl2, splits, w.part_o, w.part_ml);
+        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, idx, l.topk, H, sl2, splits, chunks, w.part_o,
+        w.part_ml);
   else
     decode_attn_kernel<false><<<grid, (H / 16) * 32, smem, stream>>>(
-        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, nullptr, 0, H, sl2, splits, w.part_o, w.part_ml);
+        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, nullptr, 0, H, sl2, splits, chunks, w.part_o,
+        w.part_ml);
   cslc_status st = check_launch("decode_attn_kernel");
   if (st != CSLC_OK) return st;
-  decode_combine_kernel<<<dim3(H, B), kD, 0, stream>>>(w.part_o, w.part_ml, l.n_entries, l.n_max, l.topk,
-                                                       l.kind == 0, H, splits, l.out);
+  decode_combine_kernel<<<dim3(H, B), 2 * kD, 0, stream>>>(w.part_o, w.part_ml, l.n_entries, l.n_max, l.topk,
+                                                           l.kind == 0, H, splits, SPLIT * chunks, l.out);
   return check_launch("decode_combine_kernel");
 }
 
@@ -698,7 +841,7 @@ cslc_status run_decode_step(const cslc_decode_layer* layers, int n_layers, int B
                             void* ws, size_t ws_bytes, cudaStream_t stream) {
   for (int i = 0; i < n_layers; ++i) {
     const cslc_decode_layer& l = layers[i];
-    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l), H);
+    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l, B), H);
     if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
     DecodeWs w;
     carve(static_cast<uint8_t*>(ws), s, w);

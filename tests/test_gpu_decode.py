@@ -133,6 +133,21 @@ def test_decode_hca_zero_and_tiny_contexts(C):
     assert_close(f64(lh.out), o_ref, rel=REL_L2_FP8, what="hca out")
 
 
+def test_decode_hca_several_chunks_per_cta(C):
+    # 4 x 157 chunks of 128 entries -> 3 chunks per attention CTA (384 entries
+    # per split): a full context, an empty one, one that ends one entry into a
+    # split's first chunk, and a ragged one
+    d = W.DecodeShape(B=4, H=64, kinds=("hca",), n_entries=(20000,))
+    n_list = [20000, 0, 385, 12345]
+    x, n = _layer_inputs(d, 0, 46, n_list)
+    lh = _gpu_layer(C, d, "hca", x, n, 1)
+    C.decode_step([lh], HI=8)
+    torch.cuda.synchronize()
+    o_ref = O.decode_hca_layer(f64(x["q"]), _oracle_kv(x), n_list, d.scale)
+    assert np.all(f64(lh.out)[1] == 0)
+    assert_close(f64(lh.out), o_ref, rel=REL_L2_FP8, what="hca out")
+
+
 def test_decode_step_is_deterministic(C):
     d = W.DecodeShape(B=2, H=64, kinds=("csa",), n_entries=(20000,))
     x, n = _layer_inputs(d, 0, 45, [20000, 12345])
