@@ -452,6 +452,13 @@ __global__ void __launch_bounds__(FIN_THREADS) decode_finalize_kernel(
 
 // -------------------------------------------------------------- attention
 
+// 2^x on the SFU (approximate; -inf gives +0, subnormal results flush to zero)
+__device__ __forceinline__ float dec_ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(r) : "f"(x));
+  return r;
+}
+
 template <bool SPARSE>
 __global__ void __launch_bounds__(256) decode_attn_kernel(
     const uint16_t* __restrict__ q, const uint8_t* __restrict__ nope, const uint16_t* __restrict__ rope,
@@ -597,7 +604,8 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
       for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const bool valid = ent[t0 + nt * 8 + 2 * tq + j] >= 0;
+          const int slot = t0 + nt * 8 + 2 * tq + j;   // within the chunk
+          const bool valid = SPARSE ? ent[slot] >= 0 : s0 + slot < n_slots;
           const float v0 = valid ? s[nt][j] * scale_log2 : -INFINITY;
           const float v1 = valid ? s[nt][2 + j] * scale_log2 : -INFINITY;
           s[nt][j] = v0;
@@ -612,7 +620,7 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
         tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
         tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
         mnew[r] = fmaxf(mrow[r], tmax[r]);
-        alpha[r] = mrow[r] == -INFINITY ? 0.f : exp2f(mrow[r] - mnew[r]);
+        alpha[r] = mrow[r] == -INFINITY ? 0.f : dec_ex2(mrow[r] - mnew[r]);
         mrow[r] = mnew[r];
       }
       float psum[2] = {0.f, 0.f};
@@ -621,7 +629,7 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int r = j >> 1;
-          const float p = mnew[r] == -INFINITY ? 0.f : exp2f(s[nt][j] - mnew[r]);
+          const float p = mnew[r] == -INFINITY ? 0.f : dec_ex2(s[nt][j] - mnew[r]);
           s[nt][j] = p;
           psum[r] += p;
         }
