@@ -478,8 +478,8 @@ def profile_case(name):
 # kernel source is the one that was measured.
 MEASURED_TRAFFIC = {
     "sparse": {"src": "sparse_attn_sm100.cu",
-               "sha256": "802c5958659538450baf7587a94be6f27bcd2214b5c8ac30757c51daabebb8ce",
-               "bytes_per_token": (172.393472e6 + 101.704960e6) / 8192},
+               "sha256": "ed29a584fc1f57bf61ff5e3eafef79629f9b0007f8da200babf5e202cc1151b0",
+               "bytes_per_token": (172.033792e6 + 102.792960e6) / 8192},
     "dense": {"src": "dense_attn_sm100.cu",
               "sha256": "af36d8a4718ffbb150d354dde250f6ce60a0ab0c0ef2dae763644e1b8e6a32e1",
               "bytes_per_token": (1.074968e9 + 1.023328e9) / 65536},
