@@ -218,10 +218,9 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
   const int n = min(n_entries[b], n_max);
   const int c0 = blockIdx.x * DEC_CHUNK;
   if (n <= topk || c0 >= n) return;
-  find_threshold_bin(ghist + (size_t)b * HIST_BINS, topk, &thr[0], &thr[1]);
-  const uint32_t T = (uint32_t)thr[0];
   const int c1 = min(n, c0 + DEC_CHUNK);
-  // this thread's scores of the chunk, all loads in flight before any is used
+  // this thread's scores of the chunk: all loads in flight before any is used,
+  // and issued before the threshold scan so that the two latencies overlap
   constexpr int PER_THREAD = DEC_CHUNK / DEC_THREADS;
   static_assert(PER_THREAD <= 16, "per-thread flags fit 16 bits");
   float sv[PER_THREAD];
@@ -230,6 +229,8 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
     const int e = c0 + i * DEC_THREADS + tid;
     sv[i] = e < c1 ? scores[(size_t)b * n_max + e] : 0.f;
   }
+  find_threshold_bin(ghist + (size_t)b * HIST_BINS, topk, &thr[0], &thr[1]);
+  const uint32_t T = (uint32_t)thr[0];
   uint32_t fa = 0u, fc = 0u;   // bit i: score i is above / inside the threshold bin
 #pragma unroll
   for (int i = 0; i < PER_THREAD; ++i) {
@@ -482,11 +483,6 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
   // chunks of this CTA that hold a slot (the rest of the split is past the end)
   const int n_chunks = slot0 >= n_slots ? 0 : min(chunks, (n_slots - slot0 + SPLIT - 1) / SPLIT);
 
-  for (int x = tid; x < H * 16; x += nthreads) {
-    const int chunk = x & 15, row = x >> 4;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)b * H + row) * kD) + chunk);
-    *reinterpret_cast<uint4*>(q_s + swz(row, chunk, 256)) = v;
-  }
   // the entries of chunk c (-1 for empty slots) into ent_buf[c & 1]
   auto fill_ent = [&](int c) {
     for (int j = tid; j < SPLIT; j += nthreads) {
@@ -520,14 +516,15 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
   };
   if (n_chunks > 0) fill_ent(0);
   __syncthreads();
-  if (n_chunks > 0) stage_chunk(0);
-  uint32_t qf[8][4];
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    const int row = warp * 16 + (lane & 15);
-    const int chunk = ks * 2 + (lane >> 4);
-    ldsm_x4(smem_u32(q_s + swz(row, chunk, 256)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+  if (n_chunks > 0) {
+    // the queries travel in the first chunk's group of copies
+    for (int x = tid; x < H * 16; x += nthreads) {
+      const int chunk = x & 15, row = x >> 4;
+      cp_async16(smem_u32(q_s + swz(row, chunk, 256)), q + ((size_t)b * H + row) * kD + chunk * 8, true);
+    }
+    stage_chunk(0);
   }
+  uint32_t qf[8][4];
   float o[16][4];
 #pragma unroll
   for (int i = 0; i < 16; ++i)
@@ -546,6 +543,14 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
       cp_async_wait<0>();
     }
     __syncthreads();
+    if (c == 0) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int row = warp * 16 + (lane & 15);
+        const int chunk = ks * 2 + (lane >> 4);
+        ldsm_x4(smem_u32(q_s + swz(row, chunk, 256)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+      }
+    }
     const int32_t* ent = ent_buf[c & 1];
     const int s0 = slot0 + c * SPLIT;
     {
