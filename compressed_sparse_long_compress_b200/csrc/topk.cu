@@ -213,7 +213,9 @@ __global__ void __launch_bounds__(TOPK_THREADS, 8) topk_rows_kernel(
   __shared__ int bcast[4];
   __shared__ int wsum[2 * TOPK_WARPS];
   __shared__ int n_cand;
-  const int r = row_begin + blockIdx.x;
+  // rows in decreasing order: the causally heaviest rows start first, so that
+  // the last wave holds the light ones
+  const int r = row_begin + (int)(gridDim.x - 1 - blockIdx.x);
   const int b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nv = n_visible((long long)q_pos0 + r, m, Nc);
