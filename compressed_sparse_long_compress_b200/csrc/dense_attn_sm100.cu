@@ -10,9 +10,13 @@
 // K (K-major) for S = Q K^T and V (MN-major) for O += P V.
 //
 // CTA roles (persistent, one CTA per SM, Q tiles in decreasing-work order):
-//   warps 0-3  softmax + epilogue, thread = row = TMEM lane. The row max is
-//              kept lazily: O (in TMEM) and the row sum are rescaled only when
-//              the max grows by more than 2^8; P goes to 128-byte-swizzled
+//   warps 0-3  softmax + epilogue, thread = row = TMEM lane. The row's
+//              reference m is the exact maximum of its first visible tile and
+//              then stays put: a later tile is redone against its exact
+//              maximum (O in TMEM and the row sum rescaled) only when its
+//              probabilities sum above 2^64, so the steady state needs no
+//              per-tile maximum (fp32 sums and bf16 P keep their relative
+//              precision at any magnitude). P goes to 128-byte-swizzled
 //              shared memory (double buffered). At the end O / l is stored.
 //   warp 4     producer: Q tile and KV tiles (TMA, STAGES-deep ring).
 //   warp 5     TMEM allocation and the single MMA-issuing thread.
@@ -36,7 +40,7 @@ constexpr int DA_ROWS = 128;
 constexpr int DA_TILE = 128;                  // entries per KV tile
 constexpr int DA_STAGES = 3;
 constexpr int DA_TILE_BYTES = DA_TILE * 256;  // 32 KB (also the Q tile and a P tile)
-constexpr float DA_GROW = 8.f;                // lazy-rescale threshold (log2 units)
+constexpr float DA_SUM_MAX = 1.8446744e19f;   // 2^64: a tile whose probabilities sum above this is redone
 
 enum { ERR_Q_EMPTY = 1, ERR_KV_EMPTY, ERR_Q_FULL, ERR_O_FREE, ERR_KV_FULL, ERR_P_FULL, ERR_S_FULL, ERR_PV_DONE,
        ERR_O_FULL, ERR_FINAL };
@@ -230,62 +234,72 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
 #pragma unroll
           for (int c = 0; c < DA_TILE; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
-        // row maximum as 8 independent chains (max is exact in any order)
-        float mx8[8];
+        // exact row maximum (scaled, log2 units); 8 independent chains
+        auto row_max = [&]() -> float {
+          float mx8[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = s[q];
+          for (int q = 0; q < 8; ++q) mx8[q] = s[q];
 #pragma unroll
-        for (int c = 8; c < DA_TILE; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        mx *= scale_log2;
-        // lazy max: move it (and rescale O, l) only when it grows by more than 2^8
-        const bool grow = mx > mrow + DA_GROW || (mrow == -INFINITY && mx != -INFINITY);
-        float alpha = 1.f;
-        if (grow) {
-          alpha = mrow == -INFINITY ? 0.f : ex2_approx(mrow - mx);
-          mrow = mx;
-          lrow *= alpha;
-        }
-        const bool warp_rescale = __any_sync(0xffffffffu, grow && alpha != 0.f && j > 0);
-        if (warp_rescale && w) {
-          if (lane == 0) w = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
-          w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
-          if (w) {
-            tc_fence_after();
+          for (int c = 8; c < DA_TILE; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+          return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+        };
+        // the row's first visible tile sets the reference (nothing to rescale yet)
+        if (mrow == -INFINITY) mrow = row_max();
+        // P = 2^(c*s - m): bf16, row-major (K-major A operand) in two 64-entry halves
+        uint8_t* prow = p_s + pb * DA_TILE_BYTES;
+        auto write_p = [&](float mneg) -> float {
+          float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent partial sums
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-              uint32_t r[32];
-              tmem_ld32(tmem + lane_off + 256 + c0, r);
-              tmem_wait_ld();
+          for (int c8 = 0; c8 < 16; ++c8) {
+            uint32_t pk[4];
 #pragma unroll
-              for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-              tmem_st32(tmem + lane_off + 256 + c0, r);
+            for (int k = 0; k < 4; ++k) {
+              const float a = ex2_approx(fmaf(s[8 * c8 + 2 * k], scale_log2, mneg));
+              const float bq = ex2_approx(fmaf(s[8 * c8 + 2 * k + 1], scale_log2, mneg));
+              ps8[2 * k] += a;
+              ps8[2 * k + 1] += bq;
+              pk[k] = pack_bf16x2(a, bq);
             }
-            tmem_wait_st();
+            *reinterpret_cast<uint4*>(prow + (c8 >> 3) * (DA_ROWS * 128) + sw128(row, c8 & 7)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          return ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        };
+        float tsum = write_p(mrow == -INFINITY ? 0.f : -mrow);
+        // a stale reference: redo the tile against its exact maximum and rescale
+        // O (after the previous PV) and l
+        const bool over = !(tsum <= DA_SUM_MAX);
+        if (__any_sync(0xffffffffu, over)) {
+          float alpha = 1.f;
+          if (over) {
+            const float mx = row_max();
+            alpha = ex2_approx(mrow - mx);
+            mrow = mx;
+            lrow *= alpha;
+            tsum = write_p(-mrow);
+          }
+          if (j > 0 && w) {
+            if (lane == 0) w = mbar_wait(&bars.pv_done, (uint32_t)((p_it - 1) & 1), abortp, errp, ERR_PV_DONE);
+            w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+            if (w) {
+              tc_fence_after();
+#pragma unroll
+              for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + 256 + c0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+                tmem_st32(tmem + lane_off + 256 + c0, r);
+              }
+              tmem_wait_st();
+            }
           }
         }
         ok = !named_bar_or(1, 128, !w || *abortp != 0);
         if (!ok) break;
-        // P = 2^(c*s - m): bf16, row-major (K-major A operand) in two 64-entry halves
-        uint8_t* prow = p_s + pb * DA_TILE_BYTES;
-        const float mneg = mrow == -INFINITY ? 0.f : -mrow;
-        float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent partial sums
-#pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float a = ex2_approx(fmaf(s[8 * c8 + 2 * k], scale_log2, mneg));
-            const float bq = ex2_approx(fmaf(s[8 * c8 + 2 * k + 1], scale_log2, mneg));
-            ps8[2 * k] += a;
-            ps8[2 * k + 1] += bq;
-            pk[k] = pack_bf16x2(a, bq);
-          }
-          *reinterpret_cast<uint4*>(prow + (c8 >> 3) * (DA_ROWS * 128) + sw128(row, c8 & 7)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-        lrow += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        lrow += tsum;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();

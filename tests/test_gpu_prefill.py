@@ -264,6 +264,32 @@ def test_dense_attention_isolated(C, H, L, m, n_c, q_pos0, q_scale):
             assert np.all(f64(out)[0, t] == 0)
 
 
+@pytest.mark.parametrize("H", [64, 16])
+def test_attention_with_scores_growing_along_the_entries(C, H):
+    # entry i scaled by 2^(i/32): the maximum of later tiles exceeds that of
+    # the first by far more than 2^64 (the references must move, O and l be
+    # rescaled), in both the dense and the sparse kernel. Outputs reach ~9e4
+    # (one bf16 ulp there is 512) and lse ~8e4, so the bounds are relative to
+    # the largest reference value.
+    L, m, n_c = 2048, 4, 512
+    q = W.randn_bf16((1, L, H, 128), 53)
+    e0 = W.randn_bf16((1, n_c, 128), 54, std=0.4).float()
+    e = (e0 * torch.exp2(torch.arange(n_c, dtype=torch.float32) / 32.0)[None, :, None]).to(torch.bfloat16)
+    scale = 1 / math.sqrt(128)
+    out, lse = C.hca_dense_attn(dev(q), dev(e), m_prime=m, scale=scale, lse=True)
+    o_ref, l_ref = O.dense_causal_attention(f64(q), f64(e), m, scale, 0)
+    assert_close_scaled(f64(out), o_ref, what="dense attn out (growing)")
+    assert_close_scaled(f64(lse), l_ref, what="dense attn lse (growing)")
+    # the sparse kernel over every visible entry of each token (ascending)
+    idx = np.full((1, L, n_c), -1, dtype=np.int32)
+    for t in range(L):
+        nv = O.n_visible(t, m, n_c)
+        idx[0, t, :nv] = np.arange(nv)
+    out_s, lse_s = C.csa_sparse_attn(dev(q), dev(e), dev(torch.from_numpy(idx)), scale, lse=True)
+    assert_close_scaled(f64(out_s), o_ref, what="sparse attn out (growing)")
+    assert_close_scaled(f64(lse_s), l_ref, what="sparse attn lse (growing)")
+
+
 def test_attention_runs_twice_identically(C):
     q = dev(W.randn_bf16((1, 300, 64, 128), 61))
     e = dev(W.randn_bf16((1, 2000, 128), 62))
