@@ -483,6 +483,7 @@ MEASURED_TRAFFIC = {
     "dense": {"src": "dense_attn_sm100.cu",
               "sha256": "73e711b1c99da856d8e4ebac26f96470f4f5e0eca29bcf506e33aa08a9f8f1f0",
               "bytes_per_token": (1.074094e9 + 1.024188e9) / 65536},
+}
 
 
 def measured_traffic(kind, tokens):
