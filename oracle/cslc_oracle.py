@@ -28,7 +28,7 @@ Sources (page title, section):
           §2.2 (compress then sparse-select), §2.3 (HCA: m' >> m, one entry per
           m' tokens, dense attention).
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
   R1 compression form: entry i, channel j is sum_t softmax_t(z_t[j] + B[s(t)][j]) * c_t[j]
      over the window tokens t, where s(t) is the token's slot in the window.
   R2 CSA window of entry i: C^b = tokens (i-1)m .. im-1 (slots 0..m-1, absent for
