@@ -290,6 +290,35 @@ def test_attention_with_scores_growing_along_the_entries(C, H):
     assert_close_scaled(f64(lse_s), l_ref, what="sparse attn lse (growing)")
 
 
+@pytest.mark.parametrize("H", [64, 128])
+def test_sparse_attention_two_sequences(C, H):
+    # B = 2: each sequence's index rows select from its own entries
+    L, n_c, topk = 150, 1500, 600
+    q = W.randn_bf16((2, L, H, 128), 71)
+    e = W.randn_bf16((2, n_c, 128), 72, std=0.4)
+    idx = np.concatenate([_random_idx(np.random.default_rng(70 + b), L, n_c, topk, holes=True) for b in range(2)])
+    scale = 1 / math.sqrt(128)
+    out, lse = C.csa_sparse_attn(dev(q), dev(e), dev(torch.from_numpy(idx)), scale, lse=True)
+    idx_ref = np.where((idx >= 0) & (idx < n_c), idx, -1)
+    o_ref, l_ref = O.sparse_attention(f64(q), f64(e), idx_ref, scale)
+    assert_close(f64(out), o_ref, what="sparse attn out (B=2)")
+    assert_close(f64(lse), l_ref, what="sparse attn lse (B=2)")
+
+
+@pytest.mark.parametrize("H,q_pos0", [(64, 0), (16, 700)])
+def test_dense_attention_two_sequences(C, H, q_pos0):
+    # B = 2 with a ragged L: the last query tile of a sequence runs past its end
+    L, m = 333, 4
+    n_c = (q_pos0 + L) // m
+    q = W.randn_bf16((2, L, H, 128), 73)
+    e = W.randn_bf16((2, n_c, 128), 74, std=0.4)
+    scale = 1 / math.sqrt(128)
+    out, lse = C.hca_dense_attn(dev(q), dev(e), m_prime=m, scale=scale, q_pos0=q_pos0, lse=True)
+    o_ref, l_ref = O.dense_causal_attention(f64(q), f64(e), m, scale, q_pos0)
+    assert_close(f64(out), o_ref, what="dense attn out (B=2)")
+    assert_close(f64(lse), l_ref, what="dense attn lse (B=2)")
+
+
 def test_attention_runs_twice_identically(C):
     q = dev(W.randn_bf16((1, 300, 64, 128), 61))
     e = dev(W.randn_bf16((1, 2000, 128), 62))
