@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
         mma_commit(&bars.o_full);
       }
       mma_commit(&bars.final_bar);
-      mbar_wait(&bars.final_bar, 0, abortp, errp, ERR_FINAL);
+      mbar_wait_done(&bars.final_bar, 0, errp, ERR_FINAL);   // also after an abort: the products finish on their own
     }
     __syncwarp();
   } else {

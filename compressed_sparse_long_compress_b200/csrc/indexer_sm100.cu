@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
         ++rq;
       }
       mma_commit(&bars.final_bar);
-      mbar_wait(&bars.final_bar, 0, abortp, errp, ERR_FINAL);
+      mbar_wait_done(&bars.final_bar, 0, errp, ERR_FINAL);   // also after an abort: the products finish on their own
     }
     __syncwarp();
   } else {

@@ -10,7 +10,12 @@
 //
 // Host code must not pass the array's name to a kernel: on the host it is only
 // a stand-in symbol. The device address is looked up once per device (with
-// that device current) through cudaGetSymbolAddress and cached.
+// that device current) through cudaGetSymbolAddress and cached together with
+// the id of the context it belongs to; when the device's context has been
+// replaced (cudaDeviceReset, or the primary context released and created
+// again) the module is loaded anew and the address is looked up again.
+
+#include <cuda.h>
 
 #include <mutex>
 
@@ -28,21 +33,52 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {0};   // id of the context the address belongs to
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 when there is none or
+// the driver cannot report it). Driver symbols are looked up once.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 }  // namespace
 
-// Device address of the static scratch on the current device (set-up on first use).
+// Device address of the static scratch on the current device (set-up on first
+// use, and again whenever the device's context has changed since).
 static cslc_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "cslc_decode_topk_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return set_error(CSLC_ERR_UNSUPPORTED, "cslc_decode_topk_noalloc: device %d", dev);
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_ctx_id();
+  if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // also makes the device's primary context current
     if (e != cudaSuccess || p == nullptr)
       return set_error(CSLC_ERR_CUDA, "cslc_decode_topk_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_ctx_id();
   }
   *out = g_noalloc_ptr[dev];
   return CSLC_OK;

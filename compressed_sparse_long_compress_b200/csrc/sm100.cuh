@@ -33,6 +33,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_test, but a thread whose phase has not completed yet is suspended
+// (it takes no issue slots) until the phase completes or about `hint_ns`
+// nanoseconds have passed.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
@@ -40,6 +52,7 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far beyond any legitimate wait
+constexpr uint32_t kSleepHintNs = 200000;          // a waiting thread re-checks the abort flag every <= 0.2 ms
 
 // Waits for the phase of `bar` with the given parity to complete. Gives up
 // after kWaitLimitNs or as soon as another role raised *abort; on giving up
@@ -49,7 +62,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_test_sleep(bar, parity, kSleepHintNs)) return true;
     if (*abort) return false;
     if (global_ns() - t0 > kWaitLimitNs) {
       *abort = 1;
@@ -57,6 +70,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// Waits (time-bounded, ignoring the abort flag) for work that completes on
+// its own -- tensor-core products or TMA copies already issued -- before the
+// CTA releases what they use. Records `code` in *err on a timeout.
+__device__ __forceinline__ bool mbar_wait_done(uint64_t* bar, uint32_t parity, int* err, int code) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_test_sleep(bar, parity, kSleepHintNs)) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(err, 0, code);
+      return false;
+    }
+  }
+  return true;
 }
 
 // ------------------------------------------------------------- fences
@@ -135,6 +162,29 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Warp-converged forms: the whole warp executes the call and one elected lane
+// (the same lane every time while the warp is converged) issues the product
+// or the commit, so the warp never diverges around the tensor-core issue.
+__device__ __forceinline__ void mma_bf16_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_increase() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_decrease() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N)); }
+
 // ------------------------------------------------------------ TMEM ld/st
 
 // 32 lanes x 32 columns of 32-bit: lane i of the warp reads row (base lane + i),
@@ -205,6 +255,19 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
 }
+// Bulk (non-tensor) copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from shared to global memory, tracked by the thread's bulk group.
+__device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(gdst), "r"(smem_u32(ssrc)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Waits until the thread's bulk copies have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// Waits until the thread's bulk copies have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
     int kv_it = 0;
     bool ok = true;
     long long tk = 0;
+    long long q_issued0 = -1, q_issued1 = -1;   // last token whose Q load went to buffer 0 / 1
     if (p == 0) tma_prefetch_map(&tm_q);
     for (long long g = blockIdx.x; g < n_tok && ok; g += gridDim.x, ++tk) {
       const int qb = (int)(tk & 1);
@@ -189,14 +190,19 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         ok = !named_bar_or(1, SA_NPROD, !w);
         if (!ok) break;
       }
+      // the index row: every element's copy in flight at once, then each
+      // thread checks its own elements (out-of-range indices become -1)
       const int32_t* irow = idx + g * (long long)topk;
       int32_t* is = idx_s + qb * SA_MAXK;
+      const uint32_t is_u = smem_u32(is);
+      for (int s = p; s < topk; s += SA_NPROD) cp_async4(is_u + 4u * s, irow + s, true);
+      cp_async_wait_all();
       int last = 0, first = SA_MAXK;
       for (int s = p; s < topk; s += SA_NPROD) {
-        int e = __ldg(irow + s);
-        if (e < 0 || e >= Nc) e = -1;
-        is[s] = e;
-        if (e >= 0) {
+        const int e = is[s];
+        if (e < 0 || e >= Nc) {
+          is[s] = -1;
+        } else {
           last = s + 1;
           first = min(first, s);
         }
@@ -216,6 +222,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         mbar_arrive_expect_tx(&bars.tok_full[qb], (uint32_t)(H * 256));
         tma_load_2d(qd, &tm_q, 0, (int)(g * H), &bars.tok_full[qb]);
         tma_load_2d(qd + SA_NP * 128, &tm_q, 64, (int)(g * H), &bars.tok_full[qb]);
+        if (qb == 0) q_issued0 = tk; else q_issued1 = tk;
       }
       const uint16_t* kvb = kv + (g / L) * (long long)Nc * kD;
       for (int j = 0; j < nt; ++j) {
@@ -246,6 +253,12 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
       }
     }
     cp_async_wait<0>();
+    // Q loads still in flight after an abort land before the CTA leaves (the
+    // last load into each buffer is the latest phase of its barrier)
+    if (p == 0) {
+      if (q_issued0 >= 0) mbar_wait_done(&bars.tok_full[0], (uint32_t)((q_issued0 >> 1) & 1), errp, ERR_TOK_FULL);
+      if (q_issued1 >= 0) mbar_wait_done(&bars.tok_full[1], (uint32_t)((q_issued1 >> 1) & 1), errp, ERR_TOK_FULL);
+    }
   } else if (warp < 8) {
     // ------------------------------------------------------ softmax + epilogue
     const int q4 = warp & 3, hh = warp >> 2;
@@ -534,9 +547,10 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         if (nt > 0 && !issue_pv(stage_1, nt - 1, ob)) { ok = false; break; }
         mma_commit(&bars.o_full[ob]);
       }
-      // every MMA issued so far has completed before TMEM is released
+      // every MMA issued so far has completed before TMEM is released, also
+      // after an abort (the products finish on their own)
       mma_commit(&bars.final_bar);
-      mbar_wait(&bars.final_bar, 0, abortp, errp, ERR_FINAL);
+      mbar_wait_done(&bars.final_bar, 0, errp, ERR_FINAL);
     }
     __syncwarp();
   }

@@ -17,7 +17,10 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
  *     never allocates or frees device memory. Scratch memory comes from a
  *     caller-provided workspace whose size the matching *_workspace_bytes()
- *     function reports (returns 0 when none is needed).
+ *     function reports (returns 0 when none is needed). One exception: the
+ *     library's module holds a static 16 MiB device array on every device
+ *     where it is loaded, until the process exits; only
+ *     cslc_decode_topk_noalloc (at the end of this header) uses it.
  *   - Tensors are dense, row-major (last index fastest) with the shapes given
  *     below. bf16 tensors are passed as cslc_bf16 (raw bfloat16 bits).
  *     Every pointer must be 16-byte aligned (CSLC_ERR_ALIGN otherwise).
@@ -239,10 +242,14 @@ cslc_status cslc_decode_topk(const float* scores, const int32_t* n_entries, int 
  * every GPU that loads the library until the process exits. The call
  * allocates nothing.
  *   - Requires cslc_decode_topk_workspace_bytes(B, n_max, topk) <= 16 MiB
- *     (e.g. B = 8 with n_max up to ~245,000); larger calls return
- *     CSLC_ERR_WORKSPACE without launching anything.
+ *     (16,777,216 bytes): e.g. B = 8 with n_max up to 259,068, or B = 64 with
+ *     n_max up to 29,695; larger calls return CSLC_ERR_WORKSPACE without
+ *     launching anything. The 1M-context shape B = 8 x 262,144 entries is over
+ *     the limit: use cslc_decode_topk with a workspace for it.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     After the device's context is replaced (cudaDeviceReset) the next call
+ *     looks the address up again, so it too must come before any capture.
  *   - Every call shares the array and it keeps the last call's contents (the
  *     parts that must start at zero are cleared on the stream by each call);
  *     calls whose work overlaps on the GPU (e.g. on two streams at once) race.

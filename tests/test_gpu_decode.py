@@ -10,7 +10,7 @@ import torch
 
 import oracle as O
 from compressed_sparse_long_compress_b200 import workloads as W
-from tests.helpers import REL_L2_FP8, assert_close, assert_close_scaled, f64
+from tests.helpers import REL_L2_FP8, assert_close, check_selection, f64, max_differing
 
 pytestmark = pytest.mark.gpu
 
@@ -70,27 +70,29 @@ def _gpu_layer(C, d, kind, x, n, topk, want_scores=True):
 
 
 def _check_csa_layer(layer, x, n_list, topk, kv_hat, seqs=None):
+    """Scores within max-abs 2e-2 / rel-L2 1e-2 of the oracle; the selection
+    exactly the top-k of the kernel's own scores; the oracle's own selection
+    identical but for verified near-ties (at most 1 % of the sequences, at
+    least one); the output equal (FP8 tolerance) to the oracle's attention over
+    the selection the kernel made, for every sequence."""
     B = len(n_list)
     seqs = range(B) if seqs is None else seqs
     sc = f64(layer.scores_out)
     idx = layer.idx_out.cpu().numpy()
     out = f64(layer.out)
     s_ref = O.decode_indexer_scores(f64(x["q_idx"]), f64(x["w"]), f64(x["k_idx"]), n_list)
-    n_same = 0
+    n_diff = 0
     for b in seqs:
         n = n_list[b]
-        assert_close_scaled(sc[b, :n], s_ref[b, :n], what=f"scores seq {b}")
+        assert_close(sc[b, :n], s_ref[b, :n], what=f"scores seq {b}")
         # the selection is exactly the top-k of the kernel's own scores
         assert np.array_equal(idx[b], O.topk_select_row(sc[b], n, topk)), b
         ref_idx = O.topk_select_row(s_ref[b], n, topk)
-        if np.array_equal(idx[b], ref_idx):
-            n_same += 1
-            sel = ref_idx[ref_idx >= 0]
-            o_ref, _ = O.attend(f64(x["q"])[b], kv_hat[b, sel], layer.scale)
-            assert_close(out[b], O.round_bf16(o_ref), rel=REL_L2_FP8, what=f"csa out seq {b}")
-        else:   # near-tie at the threshold: the sets still overlap almost fully
-            assert len(np.intersect1d(idx[b], ref_idx)) >= 0.99 * min(topk, n)
-    assert n_same >= 0.75 * len(list(seqs))
+        n_diff += not check_selection(idx[b], ref_idx, s_ref[b], n, topk)
+        sel = idx[b][idx[b] >= 0]
+        o_ref, _ = O.attend(f64(x["q"])[b], kv_hat[b, sel], layer.scale)
+        assert_close(out[b], O.round_bf16(o_ref), rel=REL_L2_FP8, what=f"csa out seq {b}")
+    assert n_diff <= max_differing(len(list(seqs))), n_diff
 
 
 def test_decode_small_csa_and_hca_layers(C):
@@ -171,7 +173,8 @@ def test_decode_full_size_sampled(C, name):
         layers.append(_gpu_layer(C, d, kind, x, n, d.topk))
     C.decode_step(layers, HI=d.HI)
     torch.cuda.synchronize()
-    seqs = [0, d.B - 1]
+    # every sequence of the hybrid step; 16 of the 64 of the CSA decode workload
+    seqs = list(range(d.B)) if d.B <= 8 else [0, 1, 2, 3, 4, 5, 6, 7, 17, 31, 40, 47, 55, 61, 62, 63]
     for li, kind in enumerate(d.kinds):
         x = {k: v[seqs] for k, v in xs[li].items()}
         n_list = [d.n_entries[li]] * len(seqs)

@@ -16,7 +16,7 @@ import torch
 
 import oracle as O
 from compressed_sparse_long_compress_b200 import workloads as W
-from tests.helpers import assert_close, assert_close_scaled, f64, rel_l2, sample_rows
+from tests.helpers import assert_close, assert_close_scaled, check_selection, f64, max_differing, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -112,15 +112,16 @@ def test_indexer_topk_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
     n_c = x["k_idx"].shape[1]
     ref_s = O.indexer_scores(f64(x["q_idx"]), f64(x["w"]), f64(x["k_idx"]), m, q_pos0)
     vis = np.isfinite(ref_s)
-    assert_close_scaled(np.where(vis, sc, -np.inf), ref_s, what="indexer scores")
+    assert_close(np.where(vis, sc, -np.inf), ref_s, what="indexer scores")
     # the selection is exactly the top-k of the scores the kernel produced
     ref_on_gpu_scores = O.topk_select(np.where(vis, sc, -np.inf), m, topk, q_pos0)
     assert np.array_equal(idx, ref_on_gpu_scores)
     assert np.array_equal(idx, idx_blocked)
     # and agrees with the oracle's own end-to-end selection up to near-ties
     ref_idx = O.topk_select(ref_s, m, topk, q_pos0)
-    same = np.mean([np.array_equal(idx[b, t], ref_idx[b, t]) for b in range(B) for t in range(L)])
-    assert same > 0.97
+    n_diff = sum(not check_selection(idx[b, t], ref_idx[b, t], ref_s[b, t], O.n_visible(q_pos0 + t, m, n_c), topk)
+                 for b in range(B) for t in range(L))
+    assert n_diff <= max_differing(B * L), n_diff
     # bit-exact visibility: count of valid slots is min(k, n_vis) and all < n_vis
     for t in range(L):
         nv = O.n_visible(q_pos0 + t, m, n_c)
@@ -352,9 +353,13 @@ def test_tiny_workload_end_to_end(C):
     assert_close(f64(e), e_ref, what="csa entries")
     assert_close(f64(eh), eh_ref, what="hca entries")
     idx = idx.cpu().numpy()
-    same = np.array([np.array_equal(idx[0, t], idx_ref[0, t]) for t in range(s.L)])
-    assert same.mean() > 0.97
+    same = np.array([check_selection(idx[0, t], idx_ref[0, t], s_ref[0, t], O.n_visible(t, s.m, s.n_c), s.topk)
+                     for t in range(s.L)])
+    assert (~same).sum() <= max_differing(s.L), (~same).sum()
     assert_close(f64(o_csa)[:, same], o_ref[:, same], what="csa out (rows with identical selection)")
+    if (~same).any():   # near-tie rows: the oracle's attention over the GPU's own selection
+        o_own, _ = O.sparse_attention(f64(x["q"]), e_ref, idx, scale, rows=np.nonzero(~same)[0])
+        assert_close(f64(o_csa)[:, ~same], o_own, what="csa out (near-tie rows, GPU selection)")
     assert_close(f64(o_hca), oh_ref, what="hca out")
     assert np.all(f64(o_csa)[0, : s.m - 1] == 0) and np.all(f64(o_hca)[0, : sh.m - 1] == 0)
 
@@ -371,7 +376,7 @@ def test_csa_prefill_full_size_sampled(C):
     idx_s, scores = C.csa_indexer_topk(x["q_idx"], x["w"], x["k_idx"], m=s.m, topk=s.topk, scores=True)
     torch.cuda.synchronize()
     assert torch.equal(idx, idx_s)
-    rows = sample_rows(s.L, 48, seed=2001)
+    rows = sample_rows(s.L, 256, seed=2001)
     e_ref = O.compress(f64(x["c"]), f64(x["z"]), f64(x["pos_bias"]), s.m, True)
     assert_close(f64(e), e_ref, what="entries")
     qi, ww = f64(x["q_idx"]), f64(x["w"])
@@ -381,18 +386,20 @@ def test_csa_prefill_full_size_sampled(C):
         s_ref[:, r] = O.indexer_scores(qi[:, t:t + 1], ww[:, t:t + 1], k_all, s.m, q_pos0=int(t))[:, 0]
     sc = f64(scores[:, torch.as_tensor(rows, device=scores.device)])
     vis = np.isfinite(s_ref)
-    assert_close_scaled(np.where(vis, sc, -np.inf), s_ref, what="scores")
+    assert_close(np.where(vis, sc, -np.inf), s_ref, what="scores")
     g_idx = idx[:, torch.as_tensor(rows, device=idx.device)].cpu().numpy()
     for r, t in enumerate(rows):
         assert np.array_equal(g_idx[0, r], O.topk_select_row(sc[0, r], O.n_visible(int(t), s.m, s.n_c), s.topk))
     ref_idx = np.stack([O.topk_select_row(s_ref[0, r], O.n_visible(int(t), s.m, s.n_c), s.topk)
                         for r, t in enumerate(rows)])[None]
-    same = np.array([np.array_equal(g_idx[0, r], ref_idx[0, r]) for r in range(len(rows))])
-    assert same.mean() > 0.9
+    same = np.array([check_selection(g_idx[0, r], ref_idx[0, r], s_ref[0, r], O.n_visible(int(t), s.m, s.n_c), s.topk)
+                     for r, t in enumerate(rows)])
+    assert (~same).sum() <= max_differing(len(rows)), (~same).sum()
     q_rows = f64(x["q"][:, torch.as_tensor(rows, device=x["q"].device)])
-    o_ref, _ = O.sparse_attention(q_rows, e_ref, ref_idx, s.scale)
+    # every sampled row: the oracle's attention over the GPU's own (verified) selection
+    o_ref, _ = O.sparse_attention(q_rows, e_ref, g_idx, s.scale)
     o_got = f64(out[:, torch.as_tensor(rows, device=out.device)])
-    assert_close(o_got[:, same], o_ref[:, same], what="csa out")
+    assert_close(o_got, o_ref, what="csa out")
 
 
 def test_hca_prefill_full_size_sampled(C):

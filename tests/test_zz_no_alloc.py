@@ -49,6 +49,36 @@ def test_noalloc_matches_workspace_version_twice(C):
     assert torch.equal(again, C.decode_topk(scores, n, topk))
 
 
+def _largest_fitting_n_max(C, B, topk, limit=16 << 20):
+    lo, hi = 0, 1 << 22
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if C.LIB.cslc_decode_topk_workspace_bytes(B, mid, topk) <= limit:
+            lo = mid
+        else:
+            hi = mid - 1
+    return lo
+
+
+def test_noalloc_at_the_size_limit(C):
+    """The largest n_max whose scratch fits the 16 MiB array (B = 8) gives
+    exactly the workspace version's indices; one entry more is refused."""
+    B, topk = 8, 1024
+    n_max = _largest_fitting_n_max(C, B, topk)
+    assert n_max == 259068
+    n_list = [n_max, n_max - 1, 200000, 1024, 1, 0, 131071, n_max]
+    scores, n = _case(B, n_max, n_list, 1203, False)
+    ref = C.decode_topk(scores, n, topk)
+    got = C.decode_topk_noalloc(scores, n, topk)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    big = torch.zeros(B, n_max + 1, device="cuda")
+    idx = torch.empty(B, topk, dtype=torch.int32, device="cuda")
+    st = C.LIB.cslc_decode_topk_noalloc(ctypes.c_void_p(big.data_ptr()), ctypes.c_void_p(n.data_ptr()), B, n_max + 1,
+                                        topk, ctypes.c_void_p(idx.data_ptr()), None)
+    assert st == 5
+
+
 def test_noalloc_rejects_oversized_calls(C):
     scores = torch.zeros(64, 40000, device="cuda")
     n = torch.full((64,), 40000, dtype=torch.int32, device="cuda")
