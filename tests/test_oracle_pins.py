@@ -1,4 +1,4 @@
-"""Pins of the CPU oracle to things other than itself (CPU only).
+"""Pins of the CPU oracles to things other than themselves (CPU only).
 
 Each test checks an oracle function against a closed form, a special case that
 reduces to a library routine (torch float64 matmul / scaled_dot_product_attention
@@ -14,9 +14,17 @@ import pytest
 import torch
 import torch.nn.functional as F
 
-import oracle as O
+import oracle as NUMPY_ORACLE
+from oracle import cpp_oracle as CPP_ORACLE
 
 RNG = np.random.default_rng(12345)
+
+
+@pytest.fixture(params=["numpy", "cpp"])
+def O(request):
+    """Every pin runs against both oracles: the float64 numpy one and the
+    float64 C++ / OpenMP one (neither is pinned by the other)."""
+    return NUMPY_ORACLE if request.param == "numpy" else CPP_ORACLE
 
 
 def bf16_values(shape, std=1.0, rng=RNG):
@@ -26,7 +34,7 @@ def bf16_values(shape, std=1.0, rng=RNG):
 
 # ---------------------------------------------------------------- rounding ---
 
-def test_round_bf16_matches_torch_cast_for_float32_inputs():
+def test_round_bf16_matches_torch_cast_for_float32_inputs(O):
     x = np.concatenate([
         RNG.standard_normal(20000) * 10.0 ** RNG.integers(-30, 30, 20000),
         np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 2.0 ** -130, 3.3e38, 3.4e38]),
@@ -36,7 +44,7 @@ def test_round_bf16_matches_torch_cast_for_float32_inputs():
     np.testing.assert_array_equal(got, ref)
 
 
-def test_round_bf16_ties_to_even_closed_form():
+def test_round_bf16_ties_to_even_closed_form(O):
     # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties to the even mantissa (1.0)
     assert O.round_bf16(np.array([1 + 2 ** -8]))[0] == 1.0
     assert O.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
@@ -45,7 +53,7 @@ def test_round_bf16_ties_to_even_closed_form():
 
 # ---------------------------------------------------------------- geometry ---
 
-def test_visibility_closed_form():
+def test_visibility_closed_form(O):
     # an entry is visible once its whole window has ended: (i+1)m - 1 <= p
     m, n_c = 4, 10
     assert [O.n_visible(p, m, n_c) for p in range(0, 12)] == [0, 0, 0, 1, 1, 1, 1, 2, 2, 2, 2, 3]
@@ -57,7 +65,7 @@ def test_visibility_closed_form():
         assert O.n_visible(p, m, n_c) == brute
 
 
-def test_window_membership():
+def test_window_membership(O):
     t, s, prev = O.compression_window(0, 4, True)
     assert list(t) == [0, 1, 2, 3] and list(s) == [4, 5, 6, 7] and not prev.any()
     t, s, prev = O.compression_window(3, 4, True)
@@ -69,7 +77,7 @@ def test_window_membership():
 
 # ------------------------------------------------------------- compressor ---
 
-def test_compression_weights_sum_to_one():
+def test_compression_weights_sum_to_one(O):
     zw = RNG.standard_normal((3, 8, 16)) * 5
     bias = RNG.standard_normal((8, 16))
     w = O.compression_weights(zw, bias)
@@ -78,7 +86,7 @@ def test_compression_weights_sum_to_one():
 
 
 @pytest.mark.parametrize("m,overlap", [(4, True), (128, False), (2, True), (3, False)])
-def test_constant_input_stays_constant(m, overlap):
+def test_constant_input_stays_constant(O, m, overlap):
     B, L, D = 2, 8 * m + 3, 16
     const = bf16_values((1, 1, D))
     c = np.broadcast_to(const, (B, L, D)).copy()
@@ -88,7 +96,7 @@ def test_constant_input_stays_constant(m, overlap):
     np.testing.assert_array_equal(e, np.broadcast_to(const, e.shape))
 
 
-def test_output_inside_window_range():
+def test_output_inside_window_range(O):
     m, B, L, D = 4, 1, 64, 32
     c, z = bf16_values((B, L, D)), bf16_values((B, L, D)) * 3
     bias = bf16_values((2 * m, D), std=0.1)
@@ -99,7 +107,7 @@ def test_output_inside_window_range():
         assert np.all(e[:, i] >= lo - 1e-12) and np.all(e[:, i] <= hi + 1e-12)
 
 
-def test_zero_logits_give_window_mean_csa():
+def test_zero_logits_give_window_mean_csa(O):
     # z = 0, bias = 0: every weight is 1/|window| -> plain mean of the window's c
     m, B, L, D = 4, 2, 40, 8
     c = bf16_values((B, L, D))
@@ -110,7 +118,7 @@ def test_zero_logits_give_window_mean_csa():
         np.testing.assert_allclose(e[:, i], c[:, (i - 1) * m:(i + 1) * m].mean(axis=1), atol=1e-14)
 
 
-def test_zero_logits_give_window_mean_hca():
+def test_zero_logits_give_window_mean_hca(O):
     m, B, L, D = 128, 1, 128 * 3 + 5, 4
     c = bf16_values((B, L, D))
     e = O.compress(c, np.zeros((B, L, D)), np.zeros((m, D)), m, False, round_output=False)
@@ -119,14 +127,14 @@ def test_zero_logits_give_window_mean_hca():
         np.testing.assert_allclose(e[:, i], c[:, i * m:(i + 1) * m].mean(axis=1), atol=1e-14)
 
 
-def test_hand_worked_example_csa_m2():
+def test_hand_worked_example_csa_m2(O):
     # D = 1, c = 1..6, z = 0, bias = 0, m = 2 (windows of 2m = 4 tokens, entry 0 only C^a)
     c = np.arange(1.0, 7.0).reshape(1, 6, 1)
     e = O.compress(c, np.zeros_like(c), np.zeros((4, 1)), 2, True, round_output=False)
     np.testing.assert_allclose(e[0, :, 0], [1.5, 2.5, 4.5], atol=1e-15)
 
 
-def test_hand_worked_example_log_weights():
+def test_hand_worked_example_log_weights(O):
     # softmax of log(a) is a / sum(a): HCA m'=3, c = 1..6, z = log([1,3,1, 2,2,4])
     c = np.arange(1.0, 7.0).reshape(1, 6, 1)
     z = np.log(np.array([1.0, 3.0, 1.0, 2.0, 2.0, 4.0])).reshape(1, 6, 1)
@@ -134,7 +142,7 @@ def test_hand_worked_example_log_weights():
     np.testing.assert_allclose(e[0, :, 0], [(1 + 6 + 3) / 5, (8 + 10 + 24) / 8], atol=1e-14)
 
 
-def test_log_weights_give_weighted_average():
+def test_log_weights_give_weighted_average(O):
     m, B, L, D = 4, 1, 32, 8
     c = bf16_values((B, L, D))
     a = RNG.uniform(0.1, 3.0, (B, L, D))
@@ -148,7 +156,7 @@ def test_log_weights_give_weighted_average():
 
 
 @pytest.mark.parametrize("overlap,m", [(True, 4), (False, 8)])
-def test_spike_selects_the_token(overlap, m):
+def test_spike_selects_the_token(O, overlap, m):
     # a huge logit on token t, channel j makes every window holding t output c_t[j]
     B, L, D = 1, 8 * m, 4
     c = bf16_values((B, L, D))
@@ -165,7 +173,7 @@ def test_spike_selects_the_token(overlap, m):
                 np.testing.assert_allclose(e[0, i, 1], c[0, toks, 1].mean(), atol=1e-14)
 
 
-def test_positional_bias_slots():
+def test_positional_bias_slots(O):
     # a huge bias on slot s picks the token in that slot: C^b slots 0..m-1, C^a m..2m-1
     m, B, L, D = 4, 1, 24, 2
     c = bf16_values((B, L, D))
@@ -181,7 +189,7 @@ def test_positional_bias_slots():
             np.testing.assert_allclose(e[0, i], c[0, tok], atol=1e-20)
 
 
-def test_separate_prev_stream():
+def test_separate_prev_stream(O):
     m, B, L, D = 4, 1, 20, 4
     c, cb = bf16_values((B, L, D)), bf16_values((B, L, D))
     zero = np.zeros((B, L, D))
@@ -192,7 +200,7 @@ def test_separate_prev_stream():
         np.testing.assert_allclose(e[:, i], ref, atol=1e-14)
 
 
-def test_m1_is_identity():
+def test_m1_is_identity(O):
     B, L, D = 2, 37, 16
     c, z = bf16_values((B, L, D)), bf16_values((B, L, D))
     e = O.compress(c, z, bf16_values((1, D), std=0.1), 1, False)
@@ -201,7 +209,7 @@ def test_m1_is_identity():
 
 # ----------------------------------------------------------------- indexer ---
 
-def test_indexer_single_head_is_relu_gemm():
+def test_indexer_single_head_is_relu_gemm(O):
     B, L, n_c, dI, m = 2, 40, 10, 64, 4
     q = bf16_values((B, L, 1, dI))
     k = bf16_values((B, n_c, dI))
@@ -213,7 +221,7 @@ def test_indexer_single_head_is_relu_gemm():
         assert np.all(np.isneginf(s[:, t, nv:]))
 
 
-def test_indexer_head_weighting():
+def test_indexer_head_weighting(O):
     B, L, n_c, HI, dI, m = 1, 32, 8, 4, 64, 4
     q = bf16_values((B, L, HI, dI))
     k = bf16_values((B, n_c, dI))
@@ -228,7 +236,7 @@ def test_indexer_head_weighting():
         np.testing.assert_allclose(s[:, t, :nv], ref[:, t, :nv], rtol=1e-6, atol=1e-6)
 
 
-def test_indexer_hand_example():
+def test_indexer_hand_example(O):
     # q heads [1,0] and [0,1]; keys [2,-1] and [-3,4]; w = [0.5, 2]
     q = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 1, 2, 2)
     k = np.array([[2.0, -1.0], [-3.0, 4.0]]).reshape(1, 2, 2)
@@ -237,7 +245,7 @@ def test_indexer_hand_example():
     np.testing.assert_array_equal(s[0, 0], [1.0, 8.0])
 
 
-def test_indexer_q_pos0_shifts_visibility():
+def test_indexer_q_pos0_shifts_visibility(O):
     B, L, n_c, HI, dI, m = 1, 16, 12, 2, 64, 4
     q, k = bf16_values((B, L, HI, dI)), bf16_values((B, n_c, dI))
     w = RNG.uniform(0, 1, (B, L, HI))
@@ -262,7 +270,7 @@ def _dominance_topk(s, k):
     return list(found[0])
 
 
-def test_topk_brute_force_tiny():
+def test_topk_brute_force_tiny(O):
     rng = np.random.default_rng(7)
     for trial in range(200):
         n = int(rng.integers(1, 10))
@@ -274,7 +282,7 @@ def test_topk_brute_force_tiny():
         assert np.all(got[kk:] == -1)
 
 
-def test_topk_hand_example_ties():
+def test_topk_hand_example_ties(O):
     s = np.array([3.0, 5.0, 5.0, 1.0, 5.0])
     assert list(O.topk_select_row(s, 5, 2)) == [1, 2]
     assert list(O.topk_select_row(s, 5, 4)) == [0, 1, 2, 4]
@@ -282,7 +290,7 @@ def test_topk_hand_example_ties():
     assert list(O.topk_select_row(s, 0, 3)) == [-1, -1, -1]
 
 
-def test_topk_invariant_under_monotone_map():
+def test_topk_invariant_under_monotone_map(O):
     rng = np.random.default_rng(8)
     s = rng.standard_normal(300)
     a = O.topk_select_row(s, 300, 37)
@@ -293,7 +301,7 @@ def test_topk_invariant_under_monotone_map():
     assert np.array_equal(a, ref)
 
 
-def test_topk_ignores_invisible_tail():
+def test_topk_ignores_invisible_tail(O):
     s = np.array([1.0, 2.0, 3.0, 100.0, 200.0])
     assert list(O.topk_select_row(s, 3, 2)) == [1, 2]
 
@@ -304,7 +312,7 @@ def _sdpa(q, k, v, mask, scale):
     return F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale)
 
 
-def test_attend_matches_sdpa_and_logsumexp():
+def test_attend_matches_sdpa_and_logsumexp(O):
     H, D, n = 6, 32, 20
     q = bf16_values((H, D))
     kv = bf16_values((n, D))
@@ -315,7 +323,7 @@ def test_attend_matches_sdpa_and_logsumexp():
     np.testing.assert_allclose(lse, torch.logsumexp(0.3 * qt[0] @ kt[0].T, dim=1).numpy(), rtol=1e-12)
 
 
-def test_attend_hand_example():
+def test_attend_hand_example(O):
     # scale 1, one head q = [1], entries [0] and [ln 3]: p = [1/4, 3/4]
     o, lse = O.attend(np.array([[1.0]]), np.array([[0.0], [math.log(3)]]), 1.0)
     assert abs(o[0, 0] - 0.75 * math.log(3)) < 1e-15
@@ -324,7 +332,7 @@ def test_attend_hand_example():
     assert np.all(o == 0) and np.all(np.isneginf(lse))
 
 
-def test_m1_hca_is_plain_causal_attention():
+def test_m1_hca_is_plain_causal_attention(O):
     # m = 1 without overlap: entries are the tokens' c, visibility is p >= i
     B, L, H, D = 1, 24, 4, 32
     c, z, q = bf16_values((B, L, D)), bf16_values((B, L, D)), bf16_values((B, L, H, D))
@@ -337,7 +345,7 @@ def test_m1_hca_is_plain_causal_attention():
     np.testing.assert_array_equal(o, O.round_bf16(ref))
 
 
-def test_sparse_attention_matches_masked_sdpa():
+def test_sparse_attention_matches_masked_sdpa(O):
     B, L, H, D, n_c, k = 1, 16, 4, 32, 12, 5
     q, e = bf16_values((B, L, H, D)), bf16_values((B, n_c, D))
     rng = np.random.default_rng(3)
@@ -355,7 +363,7 @@ def test_sparse_attention_matches_masked_sdpa():
     np.testing.assert_array_equal(o, O.round_bf16(ref))
 
 
-def test_csa_with_k_covering_all_equals_dense():
+def test_csa_with_k_covering_all_equals_dense(O):
     m, B, L, H, D, HI = 4, 1, 64, 4, 32, 2
     c, z, q = bf16_values((B, L, D)), bf16_values((B, L, D)), bf16_values((B, L, H, D))
     qi, k = bf16_values((B, L, HI, 64)), bf16_values((B, L // m, 64))
@@ -371,7 +379,7 @@ def test_csa_with_k_covering_all_equals_dense():
     assert np.all(o1[:, : m - 1] == 0)
 
 
-def test_causality_of_full_csa_pipeline():
+def test_causality_of_full_csa_pipeline(O):
     m, B, L, H, D, HI, k = 4, 1, 48, 2, 16, 2, 3
     g = np.random.default_rng(11)
     c, z, q = bf16_values((B, L, D), rng=g), bf16_values((B, L, D), rng=g), bf16_values((B, L, H, D), rng=g)
@@ -404,7 +412,7 @@ def test_causality_of_full_csa_pipeline():
 
 # ---------------------------------------------------------------- FP8 e4m3 ---
 
-def test_e4m3_decode_matches_torch_float8():
+def test_e4m3_decode_matches_torch_float8(O):
     codes = np.arange(256, dtype=np.uint8)
     ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
     got = O.e4m3_decode(codes)
@@ -412,7 +420,7 @@ def test_e4m3_decode_matches_torch_float8():
     np.testing.assert_array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
 
 
-def test_e4m3_spec_values():
+def test_e4m3_spec_values(O):
     # OCP FP8 E4M3: max normal 448 = S.1111.110, min normal 2^-6, min subnormal 2^-9
     assert O.e4m3_decode(np.array([0x7E]))[0] == 448.0
     assert O.e4m3_decode(np.array([0x08]))[0] == 2.0 ** -6
@@ -421,7 +429,7 @@ def test_e4m3_spec_values():
     assert O.e4m3_encode(np.array([1000.0, -1e9, 464.0, 0.0, -0.0]))[:5].tolist() == [0x7E, 0xFE, 0x7E, 0x00, 0x80]
 
 
-def test_e4m3_roundtrip_and_rne_vs_torch():
+def test_e4m3_roundtrip_and_rne_vs_torch(O):
     codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
     np.testing.assert_array_equal(O.e4m3_encode(O.e4m3_decode(codes)), codes)
     x = np.concatenate([RNG.standard_normal(50000) * 10.0 ** RNG.uniform(-4, 2.6, 50000),
@@ -431,13 +439,13 @@ def test_e4m3_roundtrip_and_rne_vs_torch():
     np.testing.assert_array_equal(O.e4m3_encode(x.astype(np.float64)), ref)
 
 
-def test_e4m3_relative_error_bound():
+def test_e4m3_relative_error_bound(O):
     x = RNG.uniform(2.0 ** -6, 448.0, 100000) * np.sign(RNG.standard_normal(100000))
     r = O.e4m3_decode(O.e4m3_encode(x))
     assert np.max(np.abs(r - x) / np.abs(x)) <= 2.0 ** -4
 
 
-def test_quantize_kv_mixed():
+def test_quantize_kv_mixed(O):
     e = bf16_values((3, 50, 128))
     e[1, 7] = 0.0
     codes, rope, scale = O.quantize_kv_mixed(e)
@@ -457,7 +465,7 @@ def test_quantize_kv_mixed():
 
 # ------------------------------------------------------------------ decode ---
 
-def test_decode_layers_reduce_to_dense_and_library():
+def test_decode_layers_reduce_to_dense_and_library(O):
     B, N, H, D, HI = 3, 40, 4, 128, 2
     e = bf16_values((B, N, D))
     codes, rope, scale = O.quantize_kv_mixed(e)
@@ -489,3 +497,20 @@ def test_decode_layers_reduce_to_dense_and_library():
     o_c1, idx1, _ = O.decode_csa_layer(q, qi, w, k, hat, n_entries, 5, 0.1)
     np.testing.assert_array_equal(o_c1, o_c2)
     np.testing.assert_array_equal(idx1, idx2)
+
+
+def test_cpp_compact_rows_match_full_rows():
+    """The C++ oracle's compact-row mode (sampled rows' data packed, positions
+    given) equals its full-tensor mode on the same rows."""
+    q = bf16_values((1, 300, 16, 128))
+    e = bf16_values((1, 75, 128), 0.4)
+    qi = bf16_values((1, 300, 4, 64))
+    w = np.abs(bf16_values((1, 300, 4)))
+    k = bf16_values((1, 75, 64))
+    rows = np.array([0, 3, 4, 77, 150, 299])
+    o_full, l_full = CPP_ORACLE.dense_causal_attention(q, e, 4, 0.088, q_pos0=0, rows=rows)
+    o_c, l_c = CPP_ORACLE.dense_causal_attention(q[:, rows], e, 4, 0.088, q_pos0=0, rows=rows, compact=True)
+    assert np.array_equal(o_full, o_c) and np.array_equal(l_full, l_c)
+    s_full = CPP_ORACLE.indexer_scores(qi, w, k, 4, rows=rows)
+    s_c = CPP_ORACLE.indexer_scores(qi[:, rows], w[:, rows], k, 4, rows=rows, compact=True)
+    assert np.array_equal(s_full, s_c)
