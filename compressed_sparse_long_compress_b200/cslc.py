@@ -27,7 +27,7 @@ ABI_SYMBOLS = [
     "cslc_abi_version", "cslc_last_error", "cslc_sync_status", "csa_compress", "hca_compress",
     "csa_indexer_topk_workspace_bytes", "csa_indexer_topk", "csa_topk", "csa_sparse_attn",
     "hca_dense_attn", "cslc_quantize_kv_mixed", "cslc_decode_workspace_bytes", "cslc_decode_step",
-    "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc",
+    "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc", "cslc_decode_append",
 ]
 
 
@@ -71,6 +71,7 @@ def _load():
         "cslc_decode_topk_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
         "cslc_decode_topk": (c_int, [P, P, c_int, c_int, c_int, P, P, c_size_t, P]),
         "cslc_decode_topk_noalloc": (c_int, [P, P, c_int, c_int, c_int, P, P]),
+        "cslc_decode_append": (c_int, [P, P, P, P, P, P, P, c_int, c_int, c_int, P, P, P, P, P, P, P, P, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -124,6 +125,7 @@ def sync_status(stream=None):
 # ------------------------------------------------------------- compression
 
 def csa_compress(c, z, pos_bias, m: int = 4, c_b=None, z_b=None, out=None, stream=None):
+    """D = 128 (KV entries) or 64 (indexer keys)."""
     B, L, D = c.shape
     _need(c, BF16, "c"); _need(z, BF16, "z", c.shape); _need(pos_bias, BF16, "pos_bias", (2 * m, D))
     if c_b is not None:
@@ -315,3 +317,34 @@ def decode_topk_noalloc(scores, n_entries, topk: int, idx=None, stream=None):
     _need(idx, I32, "idx", (B, topk))
     _check(LIB.cslc_decode_topk_noalloc(_ptr(scores), _ptr(n_entries), B, n_max, topk, _ptr(idx), _stream(stream)))
     return idx
+
+
+class AppendState:
+    """Caller-owned state of cslc_decode_append for one layer: the ring of the
+    last W tokens' candidates / logits (and key candidates / logits)."""
+
+    def __init__(self, B: int, m: int, overlap: bool, with_keys: bool, device):
+        self.m, self.overlap = m, overlap
+        self.W = 2 * m if overlap else m
+        self.ring_c = torch.zeros(B, self.W, 128, dtype=BF16, device=device)
+        self.ring_z = torch.zeros(B, self.W, 128, dtype=BF16, device=device)
+        self.ring_kc = torch.zeros(B, self.W, 64, dtype=BF16, device=device) if with_keys else None
+        self.ring_kz = torch.zeros(B, self.W, 64, dtype=BF16, device=device) if with_keys else None
+
+
+def decode_append(state: AppendState, c, z, pos, pos_bias, nope, rope, kv_scale, n_entries, k_c=None, k_z=None,
+                  k_pos_bias=None, k_idx=None, stream=None):
+    """One appended token per sequence (see cslc_decode_append); pos [B] int32 on the device."""
+    B = c.shape[0]
+    n_max = nope.shape[1]
+    _need(c, BF16, "c", (B, 128)); _need(z, BF16, "z", (B, 128)); _need(pos, I32, "pos", (B,))
+    _need(pos_bias, BF16, "pos_bias", (state.W, 128))
+    _need(nope, U8, "nope", (B, n_max, 64)); _need(rope, BF16, "rope", (B, n_max, 64))
+    _need(kv_scale, F32, "kv_scale", (B, n_max)); _need(n_entries, I32, "n_entries", (B,))
+    if k_c is not None:
+        _need(k_c, BF16, "k_c", (B, 64)); _need(k_z, BF16, "k_z", (B, 64))
+        _need(k_pos_bias, BF16, "k_pos_bias", (state.W, 64)); _need(k_idx, BF16, "k_idx", (B, n_max, 64))
+    _check(LIB.cslc_decode_append(_ptr(c), _ptr(z), _ptr(k_c), _ptr(k_z), _ptr(pos_bias), _ptr(k_pos_bias), _ptr(pos),
+                                  B, state.m, int(state.overlap), _ptr(state.ring_c), _ptr(state.ring_z),
+                                  _ptr(state.ring_kc), _ptr(state.ring_kz), _ptr(nope), _ptr(rope), _ptr(kv_scale),
+                                  _ptr(k_idx), n_max, _ptr(n_entries), _stream(stream)))

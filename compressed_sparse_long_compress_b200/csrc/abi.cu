@@ -26,7 +26,10 @@ cslc_status check_launch(const char* what) {
 
 // kernels (defined in the other translation units)
 cslc_status launch_compress(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*,
-                            const uint16_t*, int, int, int, int, uint16_t*, cudaStream_t);
+                            const uint16_t*, int, int, int, int, int, uint16_t*, cudaStream_t);
+cslc_status launch_decode_append(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*,
+                                 const uint16_t*, const int32_t*, int, int, int, uint16_t*, uint16_t*, uint16_t*,
+                                 uint16_t*, uint8_t*, uint16_t*, float*, uint16_t*, int, int32_t*, cudaStream_t);
 cslc_status launch_quantize_kv(const uint16_t*, long long, uint8_t*, uint16_t*, float*, cudaStream_t);
 cslc_status launch_indexer_scores(const uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int,
                                   int, int, int, int, float*, int, cudaStream_t);
@@ -132,24 +135,24 @@ cslc_status csa_compress(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16
                          const cslc_bf16* z_b, const cslc_bf16* pos_bias, int B, int L, int D, int m,
                          cslc_bf16* out, cslc_stream_t stream) {
   REQUIRE(B >= 0 && L >= 0, CSLC_ERR_SHAPE, "csa_compress: negative size");
-  REQUIRE(D == kD, CSLC_ERR_UNSUPPORTED, "csa_compress: D must be 128 (got %d)", D);
+  REQUIRE(D == kD || D == kDI, CSLC_ERR_UNSUPPORTED, "csa_compress: D must be 128 or 64 (got %d)", D);
   REQUIRE(is_pow2(m) && m <= 128, CSLC_ERR_UNSUPPORTED, "csa_compress: m must be a power of two <= 128");
   REQUIRE((c_b == nullptr) == (z_b == nullptr), CSLC_ERR_NULL, "csa_compress: give both c_b and z_b or neither");
   if ((long long)B * (L / m) == 0) return CSLC_OK;
   REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(pos_bias); REQUIRE_PTR(out);
   if (c_b) { REQUIRE_PTR(c_b); REQUIRE_PTR(z_b); }
-  return launch_compress(c, z, c_b, z_b, pos_bias, B, L, m, 1, out, stream);
+  return launch_compress(c, z, c_b, z_b, pos_bias, B, L, D, m, 1, out, stream);
 }
 
 cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16* pos_bias, int B, int L,
                          int D, int m_prime, cslc_bf16* out, cslc_stream_t stream) {
   REQUIRE(B >= 0 && L >= 0, CSLC_ERR_SHAPE, "hca_compress: negative size");
-  REQUIRE(D == kD, CSLC_ERR_UNSUPPORTED, "hca_compress: D must be 128 (got %d)", D);
+  REQUIRE(D == kD || D == kDI, CSLC_ERR_UNSUPPORTED, "hca_compress: D must be 128 or 64 (got %d)", D);
   REQUIRE(is_pow2(m_prime) && m_prime <= 128, CSLC_ERR_UNSUPPORTED,
           "hca_compress: m' must be a power of two <= 128");
   if ((long long)B * (L / m_prime) == 0) return CSLC_OK;
   REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(pos_bias); REQUIRE_PTR(out);
-  return launch_compress(c, z, nullptr, nullptr, pos_bias, B, L, m_prime, 0, out, stream);
+  return launch_compress(c, z, nullptr, nullptr, pos_bias, B, L, D, m_prime, 0, out, stream);
 }
 
 size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {
@@ -305,6 +308,30 @@ cslc_status cslc_decode_step(const cslc_decode_layer* layers, int n_layers, int 
           "cslc_decode_step: workspace of %zu bytes needed", need);
   REQUIRE(aligned16(ws), CSLC_ERR_ALIGN, "cslc_decode_step: ws is not 16-byte aligned");
   return run_decode_step(layers, n_layers, B, H, HI, ws, ws_bytes, stream);
+}
+
+cslc_status cslc_decode_append(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16* k_c, const cslc_bf16* k_z,
+                               const cslc_bf16* pos_bias, const cslc_bf16* k_pos_bias, const int32_t* pos, int B,
+                               int m, int overlap, cslc_bf16* ring_c, cslc_bf16* ring_z, cslc_bf16* ring_kc,
+                               cslc_bf16* ring_kz, uint8_t* nope, cslc_bf16* rope, float* kv_scale, cslc_bf16* k_idx,
+                               int n_max, int32_t* n_entries, cslc_stream_t stream) {
+  REQUIRE(B >= 0 && n_max >= 0, CSLC_ERR_SHAPE, "cslc_decode_append: negative size");
+  REQUIRE(is_pow2(m) && m <= 128, CSLC_ERR_UNSUPPORTED, "cslc_decode_append: m must be a power of two <= 128");
+  REQUIRE(overlap == 0 || overlap == 1, CSLC_ERR_UNSUPPORTED, "cslc_decode_append: overlap must be 0 or 1");
+  REQUIRE((k_c == nullptr) == (k_z == nullptr) && (k_c == nullptr) == (k_pos_bias == nullptr) &&
+              (k_c == nullptr) == (ring_kc == nullptr) && (k_c == nullptr) == (ring_kz == nullptr) &&
+              (k_c == nullptr) == (k_idx == nullptr),
+          CSLC_ERR_NULL, "cslc_decode_append: give all of k_c, k_z, k_pos_bias, ring_kc, ring_kz, k_idx or none");
+  if (B == 0) return CSLC_OK;
+  REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(pos_bias); REQUIRE_PTR(pos); REQUIRE_PTR(ring_c); REQUIRE_PTR(ring_z);
+  REQUIRE_PTR(n_entries);
+  if (n_max > 0) { REQUIRE_PTR(nope); REQUIRE_PTR(rope); REQUIRE_PTR(kv_scale); }
+  if (k_c) {
+    REQUIRE_PTR(k_c); REQUIRE_PTR(k_z); REQUIRE_PTR(k_pos_bias); REQUIRE_PTR(ring_kc); REQUIRE_PTR(ring_kz);
+    if (n_max > 0) REQUIRE_PTR(k_idx);
+  }
+  return launch_decode_append(c, z, k_c, k_z, pos_bias, k_pos_bias, pos, B, m, overlap, ring_c, ring_z, ring_kc,
+                              ring_kz, nope, rope, kv_scale, k_idx, n_max, n_entries, stream);
 }
 
 size_t cslc_decode_topk_workspace_bytes(int B, int n_max, int topk) {

@@ -39,37 +39,25 @@ __device__ __forceinline__ void acc_add(SoftmaxAcc& s, int j, float a, float c) 
   }
 }
 
-__global__ void __launch_bounds__(256) compress_kernel(
-    const uint16_t* __restrict__ c, const uint16_t* __restrict__ z,
-    const uint16_t* __restrict__ cb, const uint16_t* __restrict__ zb,
-    const uint16_t* __restrict__ bias, int B, int L, int m, int overlap, int n_c,
-    uint16_t* __restrict__ out) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= B * n_c) return;
-  const int b = warp / n_c;
-  const int i = warp - b * n_c;
-  const int chunk = lane & 15;
+// One compressed entry of D (128 or 64) channels, computed by one warp from
+// its W window slots; `fetch(s, cv, zv)` loads the 16-byte chunk `chunk` of
+// slot s's candidate and logit. Slots below s_begin are absent (the first CSA
+// entry has no C^b half). Every caller runs this same code, so an entry is
+// bit-identical whether it comes from a prefill pass or a decode append.
+// Lanes whose chunk lies past D / 8 compute on a valid chunk and discard it.
+template <int D, class Fetch>
+__device__ __forceinline__ void window_entry(int W, int s_begin, const uint16_t* __restrict__ bias, int lane,
+                                             Fetch fetch, float (&res)[8]) {
+  const int chunk = (lane & 15) % (D / 8);
   const int split = lane >> 4;
-
-  // Window: slots 0..W-1. CSA: slot s < m is token (i-1)m + s (C^b), slot
-  // s >= m is token i*m + s - m (C^a). HCA: slot s is token i*m + s.
-  const int W = overlap ? 2 * m : m;
   const int half = (W + 1) >> 1;
-  int s_lo = split * half, s_hi = min(W, s_lo + half);
-  if (overlap && i == 0) s_lo = max(s_lo, m);   // entry 0 has no C^b half
-
+  const int s_lo = max(split * half, s_begin), s_hi = min(W, split * half + half);
   SoftmaxAcc st;
   acc_init(st);
-  const size_t row0 = (size_t)b * L;
   for (int s = s_lo; s < s_hi; ++s) {
-    const bool prev = overlap && s < m;
-    const int t = overlap ? (i - 1) * m + s : i * m + s;
-    const uint16_t* cs = prev ? cb : c;
-    const uint16_t* zs = prev ? zb : z;
-    const uint4 cv = __ldg(reinterpret_cast<const uint4*>(cs + (row0 + t) * kD) + chunk);
-    const uint4 zv = __ldg(reinterpret_cast<const uint4*>(zs + (row0 + t) * kD) + chunk);
-    const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bias + (size_t)s * kD) + chunk);
+    uint4 cv, zv;
+    fetch(s, chunk, cv, zv);
+    const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bias + (size_t)s * D) + chunk);
     const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
     const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
     const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
@@ -80,7 +68,6 @@ __global__ void __launch_bounds__(256) compress_kernel(
     }
   }
   // merge the two halves (lanes chunk and chunk + 16)
-  float res[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float omx = __shfl_xor_sync(0xffffffffu, st.mx[j], 16);
@@ -93,26 +80,57 @@ __global__ void __launch_bounds__(256) compress_kernel(
     const float acc = st.acc[j] * f1 + oacc * f2;
     res[j] = acc / sum;
   }
-  if (split == 0) {
-    uint4 o;
-    o.x = pack_bf16x2(res[0], res[1]);
-    o.y = pack_bf16x2(res[2], res[3]);
-    o.z = pack_bf16x2(res[4], res[5]);
-    o.w = pack_bf16x2(res[6], res[7]);
-    reinterpret_cast<uint4*>(out + ((size_t)b * n_c + i) * kD)[chunk] = o;
-  }
+}
+
+__device__ __forceinline__ uint4 pack_entry_chunk(const float (&res)[8]) {
+  uint4 o;
+  o.x = pack_bf16x2(res[0], res[1]);
+  o.y = pack_bf16x2(res[2], res[3]);
+  o.z = pack_bf16x2(res[4], res[5]);
+  o.w = pack_bf16x2(res[6], res[7]);
+  return o;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) compress_kernel(
+    const uint16_t* __restrict__ c, const uint16_t* __restrict__ z,
+    const uint16_t* __restrict__ cb, const uint16_t* __restrict__ zb,
+    const uint16_t* __restrict__ bias, int B, int L, int m, int overlap, int n_c,
+    uint16_t* __restrict__ out) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= B * n_c) return;
+  const int b = warp / n_c;
+  const int i = warp - b * n_c;
+  // Window: slots 0..W-1. CSA: slot s < m is token (i-1)m + s (C^b), slot
+  // s >= m is token i*m + s - m (C^a). HCA: slot s is token i*m + s.
+  const int W = overlap ? 2 * m : m;
+  const size_t row0 = (size_t)b * L;
+  auto fetch = [&](int s, int chunk, uint4& cv, uint4& zv) {
+    const bool prev = overlap && s < m;
+    const int t = overlap ? (i - 1) * m + s : i * m + s;
+    cv = __ldg(reinterpret_cast<const uint4*>((prev ? cb : c) + (row0 + t) * D) + chunk);
+    zv = __ldg(reinterpret_cast<const uint4*>((prev ? zb : z) + (row0 + t) * D) + chunk);
+  };
+  float res[8];
+  window_entry<D>(W, overlap && i == 0 ? m : 0, bias, lane, fetch, res);
+  if (lane < D / 8) reinterpret_cast<uint4*>(out + ((size_t)b * n_c + i) * D)[lane] = pack_entry_chunk(res);
 }
 
 cslc_status launch_compress(const uint16_t* c, const uint16_t* z, const uint16_t* cb,
-                            const uint16_t* zb, const uint16_t* bias, int B, int L, int m,
+                            const uint16_t* zb, const uint16_t* bias, int B, int L, int D, int m,
                             int overlap, uint16_t* out, cudaStream_t stream) {
   const int n_c = L / m;
   const long long warps = (long long)B * n_c;
   if (warps == 0) return CSLC_OK;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  compress_kernel<<<(unsigned)blocks, threads, 0, stream>>>(c, z, cb ? cb : c, zb ? zb : z, bias,
-                                                            B, L, m, overlap, n_c, out);
+  if (D == 64)
+    compress_kernel<64><<<(unsigned)blocks, threads, 0, stream>>>(c, z, cb ? cb : c, zb ? zb : z, bias, B, L, m,
+                                                                  overlap, n_c, out);
+  else
+    compress_kernel<128><<<(unsigned)blocks, threads, 0, stream>>>(c, z, cb ? cb : c, zb ? zb : z, bias, B, L, m,
+                                                                   overlap, n_c, out);
   return check_launch("compress_kernel");
 }
 
@@ -120,6 +138,21 @@ cslc_status launch_compress(const uint16_t* c, const uint16_t* z, const uint16_t
 // Mixed decode KV layout (first page §1.4 存储格式混): dims 0..63 as e4m3 with
 // one fp32 scale per entry, dims 64..127 kept bf16. One warp per entry; lane l
 // owns dims 2l, 2l+1 of each half.
+
+// One entry's row (lane l holds dims 2l, 2l+1 in `lo` and 64+2l, 64+2l+1 in
+// `hi`) into the mixed layout; shared by the bulk quantiser and the decode
+// append so that both produce identical codes.
+__device__ __forceinline__ void quantize_row(uint32_t lo, uint32_t hi, int lane, uint8_t* __restrict__ nope_row,
+                                             uint16_t* __restrict__ rope_row, float* __restrict__ scale_out) {
+  const float x0 = bf16_lo(lo), x1 = bf16_hi(lo);
+  const float amax = warp_max(fmaxf(fabsf(x0), fabsf(x1)));
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  const float2 q = make_float2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+  const __nv_fp8x2_storage_t codes = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+  reinterpret_cast<uint16_t*>(nope_row)[lane] = codes;
+  reinterpret_cast<uint32_t*>(rope_row)[lane] = hi;
+  if (lane == 0) *scale_out = s;
+}
 
 __global__ void __launch_bounds__(256) quantize_kv_kernel(const uint16_t* __restrict__ kv,
                                                           long long n_entries,
@@ -130,16 +163,7 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(const uint16_t* __rest
   const int lane = threadIdx.x & 31;
   if (e >= n_entries) return;
   const uint32_t* row = reinterpret_cast<const uint32_t*>(kv + e * kD);
-  const uint32_t lo = row[lane];        // dims 2l, 2l+1
-  const uint32_t hi = row[32 + lane];   // dims 64+2l, 64+2l+1
-  const float x0 = bf16_lo(lo), x1 = bf16_hi(lo);
-  const float amax = warp_max(fmaxf(fabsf(x0), fabsf(x1)));
-  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-  const float2 q = make_float2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
-  const __nv_fp8x2_storage_t codes = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
-  reinterpret_cast<uint16_t*>(nope + e * kNope)[lane] = codes;
-  reinterpret_cast<uint32_t*>(rope + e * kRope)[lane] = hi;
-  if (lane == 0) scale[e] = s;
+  quantize_row(row[lane], row[32 + lane], lane, nope + e * kNope, rope + e * kRope, scale + e);
 }
 
 cslc_status launch_quantize_kv(const uint16_t* kv, long long n, uint8_t* nope, uint16_t* rope,
@@ -148,6 +172,90 @@ cslc_status launch_quantize_kv(const uint16_t* kv, long long n, uint8_t* nope, u
   const long long blocks = (n * 32 + 255) / 256;
   quantize_kv_kernel<<<(unsigned)blocks, 256, 0, stream>>>(kv, n, nope, rope, scale);
   return check_launch("quantize_kv_kernel");
+}
+
+// ---------------------------------------------------------------------------
+// Decode append ("读完这篇…" §三 压缩机制; first page §1.1 工程细节 for the
+// overlapped window): when the new token p of a sequence completes a window,
+// (p + 1) mod m == 0, entry i = (p + 1) / m - 1 is compressed from the last W
+// tokens exactly as a prefill pass would compress it, stored in the mixed
+// layout, and its indexer key is compressed the same way from the tokens'
+// 64-dim key candidates. One block per sequence: warp 0 the entry, warp 1 the
+// key. The ring holds token t in slot t mod W (W = 2m with overlap, else m).
+
+template <int D>
+__device__ __forceinline__ bool append_window(int b, int lane, int p, int m, int overlap,
+                                              const uint16_t* __restrict__ cin, const uint16_t* __restrict__ zin,
+                                              const uint16_t* __restrict__ bias, uint16_t* __restrict__ ring_c,
+                                              uint16_t* __restrict__ ring_z, int& entry, float (&res)[8]) {
+  const int W = overlap ? 2 * m : m;
+  const uint4* c_new = reinterpret_cast<const uint4*>(cin + (size_t)b * D);
+  const uint4* z_new = reinterpret_cast<const uint4*>(zin + (size_t)b * D);
+  uint16_t* rc = ring_c + (size_t)b * W * D;
+  uint16_t* rz = ring_z + (size_t)b * W * D;
+  const bool completes = (p + 1) % m == 0;
+  if (completes) {
+    const int i = (p + 1) / m - 1;
+    auto fetch = [&](int s, int chunk, uint4& cv, uint4& zv) {
+      const int t = overlap ? (i - 1) * m + s : i * m + s;
+      if (t == p) {   // the new token itself
+        cv = __ldg(c_new + chunk);
+        zv = __ldg(z_new + chunk);
+      } else {        // an earlier token, from its ring slot
+        const int slot = t % W;
+        cv = __ldg(reinterpret_cast<const uint4*>(rc + (size_t)slot * D) + chunk);
+        zv = __ldg(reinterpret_cast<const uint4*>(rz + (size_t)slot * D) + chunk);
+      }
+    };
+    window_entry<D>(W, overlap && i == 0 ? m : 0, bias, lane, fetch, res);
+    entry = i;
+  }
+  // the new token into its slot (it held token p - W, outside every window read here)
+  if (lane < D / 8) {
+    reinterpret_cast<uint4*>(rc + (size_t)(p % W) * D)[lane] = __ldg(c_new + lane);
+    reinterpret_cast<uint4*>(rz + (size_t)(p % W) * D)[lane] = __ldg(z_new + lane);
+  }
+  return completes;
+}
+
+__global__ void __launch_bounds__(64) decode_append_kernel(
+    const uint16_t* __restrict__ c, const uint16_t* __restrict__ z, const uint16_t* __restrict__ kc,
+    const uint16_t* __restrict__ kz, const uint16_t* __restrict__ bias, const uint16_t* __restrict__ kbias,
+    const int32_t* __restrict__ pos, int m, int overlap, uint16_t* __restrict__ ring_c,
+    uint16_t* __restrict__ ring_z, uint16_t* __restrict__ ring_kc, uint16_t* __restrict__ ring_kz,
+    uint8_t* __restrict__ nope, uint16_t* __restrict__ rope, float* __restrict__ kv_scale,
+    uint16_t* __restrict__ k_idx, int n_max, int32_t* __restrict__ n_entries) {
+  __shared__ uint4 row_s[kD / 8];
+  const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = pos[b];
+  if (p < 0) return;   // no new token for this sequence (uniform over the block)
+  float res[8];
+  int i = -1;
+  if (warp == 0) {
+    if (append_window<kD>(b, lane, p, m, overlap, c, z, bias, ring_c, ring_z, i, res) && i < n_max) {
+      if (lane < kD / 8) row_s[lane] = pack_entry_chunk(res);
+      __syncwarp();
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(row_s);
+      const size_t e = (size_t)b * n_max + i;
+      quantize_row(row[lane], row[32 + lane], lane, nope + e * kNope, rope + e * kRope, kv_scale + e);
+      if (lane == 0) n_entries[b] = i + 1;
+    }
+  } else if (kc != nullptr) {
+    if (append_window<kDI>(b, lane, p, m, overlap, kc, kz, kbias, ring_kc, ring_kz, i, res) && i < n_max &&
+        lane < kDI / 8)
+      reinterpret_cast<uint4*>(k_idx + ((size_t)b * n_max + i) * kDI)[lane] = pack_entry_chunk(res);
+  }
+}
+
+cslc_status launch_decode_append(const uint16_t* c, const uint16_t* z, const uint16_t* kc, const uint16_t* kz,
+                                 const uint16_t* bias, const uint16_t* kbias, const int32_t* pos, int B, int m,
+                                 int overlap, uint16_t* ring_c, uint16_t* ring_z, uint16_t* ring_kc,
+                                 uint16_t* ring_kz, uint8_t* nope, uint16_t* rope, float* kv_scale,
+                                 uint16_t* k_idx, int n_max, int32_t* n_entries, cudaStream_t stream) {
+  if (B == 0) return CSLC_OK;
+  decode_append_kernel<<<B, 64, 0, stream>>>(c, z, kc, kz, bias, kbias, pos, m, overlap, ring_c, ring_z, ring_kc,
+                                             ring_kz, nope, rope, kv_scale, k_idx, n_max, n_entries);
+  return check_launch("decode_append_kernel");
 }
 
 }  // namespace cslc

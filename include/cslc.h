@@ -91,8 +91,9 @@ cslc_status cslc_sync_status(cslc_stream_t stream);
  *                             pass both NULL to read c, z there too
  *   pos_bias  [2m, D] bf16    positional bias per window slot
  *   out       [B, floor(L/m), D] bf16
- * Requires D == 128, m a power of two in [1, 128]. L < m gives 0 entries
- * (nothing launched).
+ * Requires D == 128 (KV entries) or D == 64 (indexer keys compressed from
+ * per-token key candidates, see cslc_decode_append), m a power of two in
+ * [1, 128]. L < m gives 0 entries (nothing launched).
  */
 cslc_status csa_compress(const cslc_bf16* c, const cslc_bf16* z,
                          const cslc_bf16* c_b, const cslc_bf16* z_b,
@@ -101,7 +102,7 @@ cslc_status csa_compress(const cslc_bf16* c, const cslc_bf16* z,
 
 /* HCA compression (first page §1.2; "读完这篇…" §三 HCA 步骤简化): one window of
  * m' tokens per entry, no overlap: W_i = tokens im' .. im'+m'-1, slot = t - im'.
- *   pos_bias [m', D] bf16; out [B, floor(L/m'), D] bf16. */
+ *   pos_bias [m', D] bf16; out [B, floor(L/m'), D] bf16; D == 128 or 64. */
 cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z,
                          const cslc_bf16* pos_bias, int B, int L, int D,
                          int m_prime, cslc_bf16* out, cslc_stream_t stream);
@@ -221,6 +222,45 @@ size_t cslc_decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers
 cslc_status cslc_decode_step(const cslc_decode_layer* layers, int n_layers, int B, int H,
                              int D, int HI, int dI, void* ws, size_t ws_bytes,
                              cslc_stream_t stream);
+
+/* Decode-time incremental compression ("读完这篇…" §三 压缩机制; first page
+ * §1.1 工程细节): appends one token per sequence and, when that token completes
+ * a window, one compressed entry to the layer's decode cache.
+ *
+ * For sequence b with pos[b] = p >= 0 (the new token's absolute position;
+ * p < 0 skips the sequence): the token's c, z (and key candidate k_c, k_z) go
+ * to ring slot p mod W, W = 2m with overlap (CSA), W = m without (HCA). When
+ * (p + 1) mod m == 0, entry i = (p + 1)/m - 1 is compressed from the window of
+ * csa_compress / hca_compress (C^b = tokens (i-1)m .. im-1, C^a = im .. im+m-1;
+ * the first CSA entry has no C^b), computed by the same code as a prefill
+ * pass (bit-identical entries), stored in the mixed layout of
+ * cslc_quantize_kv_mixed at index i (bit-identical codes), its indexer key
+ * compressed the same way from the 64-dim key candidates into k_idx[b, i], and
+ * n_entries[b] = i + 1. A window completing at i >= n_max is not stored and
+ * n_entries[b] is left as it was.
+ *
+ *   c, z          [B, 128] bf16  the new token's candidate and logits
+ *   k_c, k_z      [B, 64]  bf16  its indexer-key candidate and logits, or NULL
+ *   pos_bias      [W, 128] bf16; k_pos_bias [W, 64] bf16 (NULL without keys)
+ *   pos           [B] int32 device array
+ *   ring_c/ring_z [B, W, 128], ring_kc/ring_kz [B, W, 64] bf16: caller-owned
+ *                 state; slot t mod W holds token t. Before the call it must
+ *                 hold the tokens of the window that p completes (positions
+ *                 p-W+1 .. p-1), e.g. filled by earlier appends or copied from
+ *                 a prefill's last W tokens.
+ *   nope [B, n_max, 64] u8, rope [B, n_max, 64] bf16, kv_scale [B, n_max] fp32,
+ *   k_idx [B, n_max, 64] bf16 (NULL without keys), n_entries [B] int32: the
+ *                 decode cache of cslc_decode_layer, updated in place.
+ * Requires m a power of two <= 128, overlap 0 or 1; the key arguments all
+ * given or all NULL. One launch of B blocks; no workspace.
+ */
+cslc_status cslc_decode_append(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16* k_c,
+                               const cslc_bf16* k_z, const cslc_bf16* pos_bias,
+                               const cslc_bf16* k_pos_bias, const int32_t* pos, int B, int m,
+                               int overlap, cslc_bf16* ring_c, cslc_bf16* ring_z,
+                               cslc_bf16* ring_kc, cslc_bf16* ring_kz, uint8_t* nope,
+                               cslc_bf16* rope, float* kv_scale, cslc_bf16* k_idx, int n_max,
+                               int32_t* n_entries, cslc_stream_t stream);
 
 /* The decode top-k stage alone on given scores [B, n_max] fp32: idx [B, topk]
  * = the min(topk, n_entries[b]) largest of the first n_entries[b] scores

@@ -40,8 +40,8 @@ def _err(st):
 
 
 def test_validation_unsupported_dims():
-    st, msg = _err(cslc.LIB.csa_compress(None, None, None, None, None, 1, 64, 64, 4, None, None))
-    assert st == 4 and "D must be 128" in msg
+    st, msg = _err(cslc.LIB.csa_compress(None, None, None, None, None, 1, 64, 96, 4, None, None))
+    assert st == 4 and "D must be 128 or 64" in msg
     st, msg = _err(cslc.LIB.csa_compress(None, None, None, None, None, 1, 64, 128, 3, None, None))
     assert st == 4 and "power of two" in msg
     st, _ = _err(cslc.LIB.hca_dense_attn(None, None, 1, 8, 24, 128, 4, 128, 0, 0.1, None, None, None))
@@ -86,3 +86,17 @@ def test_decode_validation():
     st, _ = _err(cslc.LIB.cslc_decode_step(arr, 1, 2, 60, 128, 8, 64, None, 0, None))
     assert st == 4   # H not a multiple of 16
     assert cslc.LIB.cslc_decode_topk_workspace_bytes(8, 262144, 1024) > 8 * 262144 * 8
+
+
+def test_validation_decode_append():
+    P = None
+    # key arguments must be all given or all NULL
+    st, msg = _err(cslc.LIB.cslc_decode_append(P, P, 16, P, P, P, P, 1, 4, 1, P, P, P, P, P, P, P, P, 8, P, P))
+    assert st == 1 and "k_c" in msg
+    st, msg = _err(cslc.LIB.cslc_decode_append(P, P, P, P, P, P, P, 1, 3, 1, P, P, P, P, P, P, P, P, 8, P, P))
+    assert st == 4 and "power of two" in msg
+    st, _ = _err(cslc.LIB.cslc_decode_append(P, P, P, P, P, P, P, 1, 4, 2, P, P, P, P, P, P, P, P, 8, P, P))
+    assert st == 4
+    st, _ = _err(cslc.LIB.cslc_decode_append(P, P, P, P, P, P, P, 2, 4, 1, P, P, P, P, P, P, P, P, 8, P, P))
+    assert st == 1   # c is NULL
+    assert cslc.LIB.cslc_decode_append(P, P, P, P, P, P, P, 0, 4, 1, P, P, P, P, P, P, P, P, 8, P, P) == 0
