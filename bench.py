@@ -537,6 +537,10 @@ def profile_case(name):
         idx = torch.empty(1, L, 1024, dtype=torch.int32, device=dev)
         for _ in range(2):   # the last 8192 query rows of a 65536-token sequence
             C.csa_indexer_topk(q_idx, w, k_idx, m=4, topk=1024, q_pos0=4 * n_c - L, scores=scores, idx=idx)
+    elif name in ("csa_decode", "hybrid_decode"):   # the full decode workloads (about 1-1.4 GB on the device)
+        wl = Decode(C, dev, 0, name)
+        for _ in range(2):
+            wl.step()
     else:
         raise SystemExit(f"unknown profile case {name}")
     torch.cuda.synchronize()
@@ -722,7 +726,8 @@ def main():
     ap.add_argument("--secondary", default="all", choices=["none", "all"])
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of timed oracle work for the headline's CPU baseline (a third for each secondary)")
-    ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192", "indexer_L8192"],
+    ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192", "indexer_L8192",
+                                                              "csa_decode", "hybrid_decode"],
                     help="run one small kernel case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:

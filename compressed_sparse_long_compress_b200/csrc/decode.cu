@@ -28,6 +28,12 @@
 //                          / PV run for all heads
 //   decode_combine_kernel  merges the splits with their max / sum statistics
 //                          (two thread groups, each over half of the splits)
+// The layers of a step are independent: layer 0 runs on the caller's stream,
+// the others on internal streams forked from it and joined back with events,
+// each with its own workspace slice. Inside a layer the kernels after the
+// first are launched as programmatic dependents: each may be scheduled while
+// its predecessor finishes and waits (griddepcontrol.wait) before it reads
+// what the predecessor wrote.
 
 #include <algorithm>
 
@@ -44,6 +50,12 @@ constexpr int ATTN_CTAS = 296;       // attention CTAs aimed at per layer: two p
 constexpr int DTILE = 64;            // entries per attention tile
 constexpr int FIN_THREADS = 1024;
 constexpr int MAX_TOPK = 2048;
+
+// Programmatic dependent launch: wait for the preceding kernel's results (a
+// no-op when the kernel was not launched as a dependent), and let the next
+// kernel be scheduled once every CTA of this one has reached this point.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 struct DecodeWs {
   float* scores;          // [B, n_max]
@@ -147,6 +159,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_scores_kernel(
     const uint32_t v = hist[x];
     if (v) atomicAdd(&gh[x], v);
   }
+  pdl_trigger();
 }
 
 // Histogram only (for the stand-alone top-k entry on given scores).
@@ -214,6 +227,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
     uint2* __restrict__ cand) {
   __shared__ int thr[2];
   const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  pdl_wait();
   if (tid == 0) { thr[0] = HIST_BINS; thr[1] = 0; }   // "nothing above" if no bin is found
   const int n = min(n_entries[b], n_max);
   const int c0 = blockIdx.x * DEC_CHUNK;
@@ -279,6 +293,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_select_kernel(
       ++pc;
     }
   }
+  pdl_trigger();
 }
 
 // 64-bit composite of a candidate: score key, then reversed index, so that a
@@ -295,6 +310,8 @@ __global__ void __launch_bounds__(FIN_THREADS) decode_finalize_kernel(
   __shared__ int bc[4];
   __shared__ int fill;
   const int b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_trigger();   // the attention's CTAs may be scheduled meanwhile (they wait for this grid)
   const int n = min(n_entries[b], n_max);
   int32_t* out = idx + (size_t)b * topk;
   if (n <= topk) {
@@ -476,6 +493,7 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
   const int b = blockIdx.y, sp = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nthreads = (H / 16) * 32;
+  pdl_wait();
   const int g = lane >> 2, tq = lane & 3;
   const int n = min(n_entries[b], n_max);
   const int n_slots = SPARSE ? topk : n;
@@ -684,6 +702,7 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(
     pm[2 * h0] = mrow[0]; pm[2 * h0 + 1] = lrow[0];
     pm[2 * h1] = mrow[1]; pm[2 * h1 + 1] = lrow[1];
   }
+  pdl_trigger();
 }
 
 __global__ void __launch_bounds__(2 * kD) decode_combine_kernel(const float* __restrict__ part_o,
@@ -694,6 +713,7 @@ __global__ void __launch_bounds__(2 * kD) decode_combine_kernel(const float* __r
                                                                 uint16_t* __restrict__ out) {
   __shared__ float xm[kD], xn[kD], xd[kD];
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x & (kD - 1), grp = threadIdx.x / kD;
+  pdl_wait();
   const int n = min(n_entries[b], n_max);
   const int slots = sparse ? min(topk, n) : n;
   const int used = min(splits, (slots + split_slots - 1) / split_slots);
@@ -748,6 +768,23 @@ __global__ void __launch_bounds__(2 * kD) decode_combine_kernel(const float* __r
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Launches `kernel` as a programmatic dependent of the work before it on `stream`.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct DecodeWsSizes {
   size_t scores, hist, counters, sel, cand, idx, part_o, part_ml;
   size_t total() const { return scores + hist + counters + sel + cand + idx + part_o + part_ml; }
@@ -778,15 +815,18 @@ static DecodeWsSizes ws_sizes(int B, int n_max, int topk, int splits, int H) {
   return s;
 }
 
+static DecodeWsSizes layer_ws_sizes(const cslc_decode_layer& l, int B, int H) {
+  DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l, B), H);
+  if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
+  return s;
+}
+
+// The layers run concurrently, so each has its own slice; the histograms and
+// counters of all layers come first, so that one memset clears them.
 size_t decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers, int B, int H) {
-  size_t best = 0;
-  for (int i = 0; i < n_layers; ++i) {
-    const cslc_decode_layer& l = layers[i];
-    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l, B), H);
-    if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
-    best = s.total() > best ? s.total() : best;
-  }
-  return best;
+  size_t total = 0;
+  for (int i = 0; i < n_layers; ++i) total += layer_ws_sizes(layers[i], B, H).total();
+  return total;
 }
 
 size_t decode_topk_workspace_bytes(int B, int n_max, int topk) {
@@ -809,14 +849,14 @@ static void carve(uint8_t* base, const DecodeWsSizes& s, DecodeWs& w) {
 static cslc_status run_topk_stages(const float* scores, const int32_t* n_entries, int B, int n_max,
                                    int topk, DecodeWs& w, int32_t* idx, cudaStream_t stream) {
   const dim3 grid((n_max + DEC_CHUNK - 1) / DEC_CHUNK, B);
-  if (n_max > 0) {
-    decode_select_kernel<<<grid, DEC_THREADS, 0, stream>>>(scores, n_entries, n_max, topk, w.hist,
-                                                           w.counters, w.sel, w.cand);
-    cslc_status st = check_launch("decode_select_kernel");
-    if (st != CSLC_OK) return st;
-  }
-  decode_finalize_kernel<<<B, FIN_THREADS, 0, stream>>>(n_entries, n_max, topk, w.counters, w.sel,
-                                                        w.cand, idx);
+  cudaError_t e = cudaSuccess;
+  if (n_max > 0)
+    e = launch_dependent(decode_select_kernel, grid, dim3(DEC_THREADS), 0, stream, scores, n_entries, n_max, topk,
+                         w.hist, w.counters, w.sel, w.cand);
+  if (e == cudaSuccess)
+    e = launch_dependent(decode_finalize_kernel, dim3(B), dim3(FIN_THREADS), 0, stream, n_entries, n_max, topk,
+                         w.counters, w.sel, w.cand, idx);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "decode top-k launch: %s", cudaGetErrorString(e));
   return check_launch("decode_finalize_kernel");
 }
 
@@ -835,35 +875,111 @@ static cslc_status run_attention(const cslc_decode_layer& l, int B, int H, const
   }
   const dim3 grid(splits, B);
   const float sl2 = l.scale * kLog2e;
-  if (l.kind == 0)
-    decode_attn_kernel<true><<<grid, (H / 16) * 32, smem, stream>>>(
-        l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, idx, l.topk, H, sl2, splits, chunks, w.part_o,
-        w.part_ml);
-  else
+  cudaError_t e;
+  if (l.kind == 0)   // after the top-k: a programmatic dependent of its finalize pass
+    e = launch_dependent(decode_attn_kernel<true>, grid, dim3((H / 16) * 32), smem, stream, l.q, l.nope, l.rope,
+                         l.kv_scale, l.n_entries, l.n_max, idx, l.topk, H, sl2, splits, chunks, w.part_o, w.part_ml);
+  else {             // the first kernel of an HCA layer: an ordinary launch
     decode_attn_kernel<false><<<grid, (H / 16) * 32, smem, stream>>>(
         l.q, l.nope, l.rope, l.kv_scale, l.n_entries, l.n_max, nullptr, 0, H, sl2, splits, chunks, w.part_o,
         w.part_ml);
-  cslc_status st = check_launch("decode_attn_kernel");
-  if (st != CSLC_OK) return st;
-  decode_combine_kernel<<<dim3(H, B), 2 * kD, 0, stream>>>(w.part_o, w.part_ml, l.n_entries, l.n_max, l.topk,
-                                                           l.kind == 0, H, splits, SPLIT * chunks, l.out);
-  return check_launch("decode_combine_kernel");
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess)
+    e = launch_dependent(decode_combine_kernel, dim3(H, B), dim3(2 * kD), 0, stream, w.part_o, w.part_ml,
+                         l.n_entries, l.n_max, l.topk, (int)(l.kind == 0), H, splits, SPLIT * chunks, l.out);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "decode attention launch: %s", cudaGetErrorString(e));
+  return CSLC_OK;
 }
+
+// Internal streams and events for the layers after the first, one set per
+// host thread and device (created on first use, kept for the process).
+constexpr int kMaxLayerStreams = 15;
+struct LayerStreams {
+  cudaStream_t s[kMaxLayerStreams] = {};
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t done[kMaxLayerStreams] = {};
+};
+
+static cslc_status layer_streams(LayerStreams** out) {
+  constexpr int kMaxDevices = 64;
+  thread_local LayerStreams sets[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return set_error(CSLC_ERR_CUDA, "cslc_decode_step: no usable current device");
+  LayerStreams& o = sets[dev];
+  if (!o.fork) {
+    e = cudaEventCreateWithFlags(&o.fork, cudaEventDisableTiming);
+    for (int j = 0; j < kMaxLayerStreams && e == cudaSuccess; ++j) {
+      e = cudaStreamCreateWithFlags(&o.s[j], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&o.done[j], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {
+      o.fork = nullptr;
+      return set_error(CSLC_ERR_CUDA, "cslc_decode_step: stream/event creation: %s", cudaGetErrorString(e));
+    }
+  }
+  *out = &o;
+  return CSLC_OK;
+}
+
+static cslc_status run_layer(const cslc_decode_layer& l, int B, int H, int HI, DecodeWs& w, cudaStream_t stream);
 
 cslc_status run_decode_step(const cslc_decode_layer* layers, int n_layers, int B, int H, int HI,
                             void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)ws_bytes;
+  if (n_layers > 1 + kMaxLayerStreams)
+    return set_error(CSLC_ERR_UNSUPPORTED, "cslc_decode_step: at most %d layers per call", 1 + kMaxLayerStreams);
+  // carve: every layer's histogram + counters, then each layer's other buffers
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t zero_bytes = 0;
   for (int i = 0; i < n_layers; ++i) {
-    const cslc_decode_layer& l = layers[i];
-    DecodeWsSizes s = ws_sizes(B, l.n_max, l.kind == 0 ? l.topk : 1, layer_splits(l, B), H);
-    if (l.kind != 0) s.scores = s.hist = s.counters = s.sel = s.cand = s.idx = 0;
-    DecodeWs w;
-    carve(static_cast<uint8_t*>(ws), s, w);
+    const DecodeWsSizes s = layer_ws_sizes(layers[i], B, H);
+    zero_bytes += s.hist + s.counters;
+  }
+  uint8_t* zp = base;
+  uint8_t* rp = base + zero_bytes;
+  DecodeWs w[1 + kMaxLayerStreams];
+  for (int i = 0; i < n_layers; ++i) {
+    const DecodeWsSizes s = layer_ws_sizes(layers[i], B, H);
+    w[i].hist = reinterpret_cast<uint32_t*>(zp); zp += s.hist;
+    w[i].counters = reinterpret_cast<int32_t*>(zp); zp += s.counters;
+    w[i].scores = reinterpret_cast<float*>(rp); rp += s.scores;
+    w[i].sel = reinterpret_cast<int32_t*>(rp); rp += s.sel;
+    w[i].cand = reinterpret_cast<uint2*>(rp); rp += s.cand;
+    w[i].idx = reinterpret_cast<int32_t*>(rp); rp += s.idx;
+    w[i].part_o = reinterpret_cast<float*>(rp); rp += s.part_o;
+    w[i].part_ml = reinterpret_cast<float*>(rp); rp += s.part_ml;
+  }
+  if (zero_bytes && cudaMemsetAsync(base, 0, zero_bytes, stream) != cudaSuccess)
+    return set_error(CSLC_ERR_CUDA, "cudaMemsetAsync failed");
+  if (n_layers == 1) return run_layer(layers[0], B, H, HI, w[0], stream);
+  LayerStreams* ls = nullptr;
+  cslc_status st = layer_streams(&ls);
+  if (st != CSLC_OK) return st;
+  cudaError_t e = cudaEventRecord(ls->fork, stream);
+  for (int i = 1; i < n_layers && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(ls->s[i - 1], ls->fork, 0);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "cslc_decode_step: %s", cudaGetErrorString(e));
+  for (int i = 0; i < n_layers; ++i) {
+    st = run_layer(layers[i], B, H, HI, w[i], i == 0 ? stream : ls->s[i - 1]);
+    if (st != CSLC_OK) return st;
+  }
+  // join: `stream` continues after every layer
+  for (int i = 1; i < n_layers && e == cudaSuccess; ++i) {
+    e = cudaEventRecord(ls->done[i - 1], ls->s[i - 1]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ls->done[i - 1], 0);
+  }
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "cslc_decode_step: %s", cudaGetErrorString(e));
+  return CSLC_OK;
+}
+
+static cslc_status run_layer(const cslc_decode_layer& l, int B, int H, int HI, DecodeWs& w, cudaStream_t stream) {
+  {
     cslc_status st;
     if (l.kind == 0) {
       float* scores = l.scores_out ? l.scores_out : w.scores;
       int32_t* idx = l.idx_out ? l.idx_out : w.idx;
-      if (cudaMemsetAsync(w.hist, 0, s.hist + s.counters, stream) != cudaSuccess)
-        return set_error(CSLC_ERR_CUDA, "cudaMemsetAsync failed");
       if (l.n_max > 0) {
         const dim3 grid((l.n_max + DEC_CHUNK - 1) / DEC_CHUNK, B);
         if (HI <= 8)
@@ -881,9 +997,8 @@ cslc_status run_decode_step(const cslc_decode_layer* layers, int n_layers, int B
     } else {
       st = run_attention(l, B, H, nullptr, w, stream);
     }
-    if (st != CSLC_OK) return st;
+    return st;
   }
-  return CSLC_OK;
 }
 
 cslc_status run_decode_topk(const float* scores, const int32_t* n_entries, int B, int n_max, int topk,

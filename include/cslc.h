@@ -211,14 +211,18 @@ typedef struct {
   float* scores_out;         /* [B, n_max] fp32 indexer scores (CSA), or NULL */
 } cslc_decode_layer;
 
-/* Workspace for cslc_decode_step over these layers (the maximum over layers;
- * layers run one after another on the stream and reuse it). */
+/* Workspace for cslc_decode_step over these layers: the sum of the layers'
+ * needs (the layers run concurrently, each on its own slice). */
 size_t cslc_decode_workspace_bytes(const cslc_decode_layer* layers, int n_layers, int B,
                                    int H, int HI);
 
-/* Runs the layers in order on `stream` (the hybrid C,H,C,H decode step is
- * four layers). Requires D == 128, d_I == 64, H a multiple of 16 <= 128,
- * 1 <= H_I <= 16. */
+/* Runs the layers (the hybrid C,H,C,H decode step is four layers, at most
+ * 16 per call). The layers are independent and run concurrently: layer 0 on
+ * `stream`, the others on internal streams (one set per host thread and
+ * device) that are forked from `stream` and joined back into it, so work
+ * queued on `stream` before the call happens before every layer and work
+ * queued after it happens after all of them (also under stream capture).
+ * Requires D == 128, d_I == 64, H a multiple of 16 <= 128, 1 <= H_I <= 16. */
 cslc_status cslc_decode_step(const cslc_decode_layer* layers, int n_layers, int B, int H,
                              int D, int HI, int dI, void* ws, size_t ws_bytes,
                              cslc_stream_t stream);
