@@ -54,6 +54,7 @@ _dequant = _sig("orc_dequantize_kv_mixed", None, [_U8, _D, _F32, _ll, _D])
 _dec_scores = _sig("orc_decode_indexer_scores", None, [_D, _D, _D, _I64, _i, _ll, _i, _i, _D])
 _dec_csa = _sig("orc_decode_csa_layer", None, [_D, _D, _D, _I64, _i, _i, _i, _ll, _i, _d, _D, _I32])
 _dec_hca = _sig("orc_decode_hca_layer", None, [_D, _D, _I64, _i, _i, _i, _ll, _d, _D])
+_project = _sig("orc_project", None, [_D, _D, _ll, _i, _i, _D])
 _threads = _sig("orc_threads", _i, [])
 _set_threads = _sig("orc_set_threads", None, [_i])
 
@@ -130,6 +131,23 @@ def compress(c, z, pos_bias, m: int, overlap: bool, c_b=None, z_b=None, round_ou
     _compress(c, z, pos_bias, None if cb is None else cb.ctypes.data_as(_P), None if zb is None else zb.ctypes.data_as(_P),
               B, L, D, m, int(bool(overlap)), int(bool(round_output)), out)
     return out
+
+
+def project(h, W):
+    h, W = _f64(h), _f64(W)
+    B, L, dm = h.shape
+    D = W.shape[0]
+    out = np.empty((B, L, D))
+    _project(h.reshape(B * L, dm), W, B * L, dm, D, out.reshape(B * L, D))
+    return out
+
+
+def compressor_front_end(h, W, pos_bias, m: int, overlap: bool, round_output: bool = True):
+    W = _f64(W)
+    if overlap:
+        return compress(project(h, W[0]), project(h, W[2]), pos_bias, m, True,
+                        c_b=project(h, W[1]), z_b=project(h, W[3]), round_output=round_output)
+    return compress(project(h, W[0]), project(h, W[1]), pos_bias, m, False, round_output=round_output)
 
 
 def csa_compress(c, z, pos_bias, m: int = 4, c_b=None, z_b=None, round_output=True):

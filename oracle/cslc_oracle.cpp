@@ -193,6 +193,18 @@ int orc_compression_window(long long i, int m, int overlap, long long* tokens, i
   return n;
 }
 
+// One learned projection of the compressor front end: out[r, n] = sum_k
+// h[r, k] W[n, k] for the rows r of h [rows, d_model] and W [D, d_model].
+void orc_project(const double* h, const double* W, long long rows, int d_model, int D, double* out) {
+#pragma omp parallel for schedule(static)
+  for (long long r = 0; r < rows; ++r)
+    for (int n = 0; n < D; ++n) {
+      double acc = 0.0;
+      for (int k = 0; k < d_model; ++k) acc += h[(size_t)r * d_model + k] * W[(size_t)n * d_model + k];
+      out[(size_t)r * D + n] = acc;
+    }
+}
+
 // Per-channel softmax over the W window tokens of (z + bias[slot]).
 // zw: [W, D]; bias_rows: [W, D]; out: [W, D].
 void orc_compression_weights(const double* zw, const double* bias_rows, int W, int D, double* out) {

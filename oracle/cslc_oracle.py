@@ -70,7 +70,7 @@ __all__ = [
     "attend", "sparse_attention", "dense_causal_attention",
     "E4M3_MAX", "e4m3_decode", "e4m3_encode", "quantize_kv_mixed",
     "dequantize_kv_mixed", "decode_indexer_scores", "decode_csa_layer",
-    "decode_hca_layer",
+    "decode_hca_layer", "project", "compressor_front_end",
 ]
 
 F64 = np.float64
@@ -181,6 +181,27 @@ def compress(c, z, pos_bias, m: int, overlap: bool, c_b=None, z_b=None,
         wts = compression_weights(zw, pos_bias[slots])
         out[:, i] = (wts * cw).sum(axis=1)
     return round_bf16(out) if round_output else out
+
+
+def project(h, W):
+    """One learned projection of the compressor front end: h [B, L, d_model]
+    times W^T for W [D, d_model] (the nn.Linear layout), in float64."""
+    return np.einsum("bld,nd->bln", np.asarray(h, dtype=F64), np.asarray(W, dtype=F64))
+
+
+def compressor_front_end(h, W, pos_bias, m: int, overlap: bool, round_output: bool = True):
+    """Compressed entries straight from hidden states ([READ] §三 压缩机制: "4 W
+    + 2 B" learnable). CSA (overlap): W [4, D, d_model] holds W^{a,KV},
+    W^{b,KV}, W^{a,Z}, W^{b,Z}; the C^a half of a window uses c = h W^{a,KV},
+    z = h W^{a,Z}, the C^b half c_b = h W^{b,KV}, z_b = h W^{b,Z}; pos_bias
+    [2m, D] holds the two B matrices (C^b slots, then C^a slots). HCA: W [2, D,
+    d_model] holds W^{KV}, W^{Z}; pos_bias [m', D]. The projections stay in
+    float64 (nothing is rounded between the projection and the compression)."""
+    W = np.asarray(W, dtype=F64)
+    if overlap:
+        return compress(project(h, W[0]), project(h, W[2]), pos_bias, m, True,
+                        c_b=project(h, W[1]), z_b=project(h, W[3]), round_output=round_output)
+    return compress(project(h, W[0]), project(h, W[1]), pos_bias, m, False, round_output=round_output)
 
 
 def csa_compress(c, z, pos_bias, m: int = 4, c_b=None, z_b=None, round_output=True):

@@ -514,3 +514,42 @@ def test_cpp_compact_rows_match_full_rows():
     s_full = CPP_ORACLE.indexer_scores(qi, w, k, 4, rows=rows)
     s_c = CPP_ORACLE.indexer_scores(qi[:, rows], w[:, rows], k, 4, rows=rows, compact=True)
     assert np.array_equal(s_full, s_c)
+
+
+# ------------------------------------------------- compressor front end ---
+
+def test_projection_is_a_float64_matmul(O):
+    h = bf16_values((2, 7, 96))
+    W = bf16_values((5, 96))
+    ref = torch.matmul(torch.from_numpy(h), torch.from_numpy(W).T).numpy()
+    assert np.allclose(O.project(h, W), ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("overlap,m", [(True, 4), (False, 8)])
+def test_front_end_with_identity_projections_is_compress(O, overlap, m):
+    """With every W the identity (d_model = D) the front end is the compressor
+    on the hidden states themselves (c = z = h, and c_b = z_b = h for CSA)."""
+    D = 16
+    h = bf16_values((1, 8 * m, D))
+    eye = np.eye(D)
+    W = np.stack([eye] * (4 if overlap else 2))
+    bias = bf16_values((2 * m if overlap else m, D), 0.1)
+    got = O.compressor_front_end(h, W, bias, m, overlap)
+    assert np.array_equal(got, O.compress(h, h, bias, m, overlap))
+
+
+def test_front_end_uses_each_projection_in_its_place(O):
+    """W^{b,*} reach only the C^b half and W^{a,*} only the C^a half: with
+    zero logit weights (uniform windows) the entry is the mean over the window
+    of h W^{b,KV} on the C^b tokens and h W^{a,KV} on the C^a tokens."""
+    m, D, dm = 4, 8, 24
+    h = bf16_values((1, 6 * m, dm))
+    Wa, Wb = bf16_values((D, dm)), bf16_values((D, dm))
+    zero = np.zeros((D, dm))
+    got = O.compressor_front_end(h, np.stack([Wa, Wb, zero, zero]), np.zeros((2 * m, D)), m, True,
+                                 round_output=False)
+    ca, cb = h[0] @ Wa.T, h[0] @ Wb.T
+    for i in range(6):
+        cur = ca[i * m:(i + 1) * m]
+        ref = cur.mean(axis=0) if i == 0 else np.concatenate([cb[(i - 1) * m:i * m], cur]).mean(axis=0)
+        assert np.allclose(got[0, i], ref, rtol=1e-12, atol=1e-12)
