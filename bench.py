@@ -273,6 +273,44 @@ class HcaPrefill:
         return workload_config(self.name)
 
 
+class FrontEnd:
+    name = "front_end_prefill"
+
+    def __init__(self, C, device, rank):
+        wl = W.WORKLOADS[self.name]
+        self.s = s = wl.front_end
+        self.C = C
+        self.x = W.front_end_inputs(s, rank_seed(wl.wid, rank), device=device)
+        self.e = torch.empty(s.B, s.n_c, 128, dtype=torch.bfloat16, device=device)
+        self.launches = 1
+        self.flops = 2.0 * s.B * s.L * s.d_model * 128 * s.n_proj   # every token through the projections once
+        self.units = s.B * s.L
+
+    def step(self, timer=None):
+        s, x = self.s, self.x
+        if timer:
+            timer[0].record()
+        self.C.compress_front_end(x["h"], x["W"], x["pos_bias"], s.m, s.overlap, out=self.e)
+        if timer:
+            timer[1].record()
+
+    def input_tensors(self):
+        return [self.x["h"], self.x["W"], self.x["pos_bias"]]
+
+    def output_tensors(self):
+        return [self.e]
+
+    def roofline(self, kernel_ms, peaks):
+        ach = self.flops / (kernel_ms * 1e-3) / 1e12
+        return {"kernel": "compress_front_end (front_end_sm100_kernel<true>)", "bound": "tensor",
+                "achieved": round(ach, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": None,
+                "algorithmic_flops_per_launch": self.flops, "peak_source": peaks["source"] + " (burst)"}
+
+    def config(self):
+        return workload_config(self.name)
+
+
 class Decode:
     def __init__(self, C, device, rank, name):
         self.name = name
@@ -336,6 +374,10 @@ def workload_config(name):
         return {"workload": "hca_prefill: HCA prefill, batch 1, L=1048576, m'=128 -> 8192 entries, 64 heads x 128, "
                             "dense causal", "global_batch": s.B, "seq_len": s.L, "heads": s.H, "m_prime": s.m,
                 "l2": "inputs larger than L2 (q 16 GiB)"}
+    if wl.front_end is not None:
+        f = wl.front_end
+        return {"workload": f"{name}: " + wl.description, "global_batch": f.B, "seq_len": f.L,
+                "d_model": f.d_model, "m": f.m, "l2": "inputs larger than L2 (h 940 MB)"}
     if wl.decode is not None:
         d = wl.decode
         return {"workload": f"{name}: " + wl.description, "global_batch": d.B, "layers": list(d.kinds),
@@ -349,6 +391,8 @@ def make_workload(name, C, device, rank):
         return CsaPrefill(C, device, rank)
     if name == "hca_prefill":
         return HcaPrefill(C, device, rank)
+    if name == "front_end_prefill":
+        return FrontEnd(C, device, rank)
     return Decode(C, device, rank, name)
 
 
@@ -537,6 +581,11 @@ def profile_case(name):
         idx = torch.empty(1, L, 1024, dtype=torch.int32, device=dev)
         for _ in range(2):   # the last 8192 query rows of a 65536-token sequence
             C.csa_indexer_topk(q_idx, w, k_idx, m=4, topk=1024, q_pos0=4 * n_c - L, scores=scores, idx=idx)
+    elif name == "front_end_L16384":   # 16384 tokens of d_model 7168 (235 MB of hidden states)
+        s = W.FrontEndShape(B=1, L=16384, d_model=7168)
+        x = W.front_end_inputs(s, 6, device=dev)
+        for _ in range(2):
+            C.compress_front_end(x["h"], x["W"], x["pos_bias"], s.m, True)
     elif name in ("csa_decode", "hybrid_decode"):   # the full decode workloads (about 1-1.4 GB on the device)
         wl = Decode(C, dev, 0, name)
         for _ in range(2):
@@ -625,6 +674,26 @@ def oracle_sample(name, budget_s=10.0, one_thread_s=0.0):
             done1, t1 = rows_batch(4, one_thread_s)
             CO.set_threads(threads)
             res["value_1thread"] = 1.0 / (t1 / done1 + t_comp1 / s.L)
+        return res
+    if name == "front_end_prefill":
+        wl = W.WORKLOADS[name]
+        s = wl.front_end
+        x = W.front_end_inputs(s, wl.wid)
+        Wt, bias = f(x["W"]), f(x["pos_bias"])
+        rng = np.random.default_rng(7)
+        done, t_e = 0, 0.0
+        while t_e < budget_s:
+            i = int(rng.integers(1, s.n_c))
+            toks = f(x["h"][:, (i - 1) * s.m:(i + 1) * s.m])
+            t1 = time.perf_counter()
+            CO.compressor_front_end(toks, Wt, bias, s.m, True)
+            t_e += time.perf_counter() - t1
+            done += 1
+        res["value"] = s.m / (t_e / done)   # every entry advances the sequence by m tokens
+        res["unit"] = "tokens/s"
+        res["sample"] = (f"C++ oracle: projections and compression of {done} uniformly drawn entries, each from its "
+                         f"own 2m = {2 * s.m}-token window ({t_e:.1f} s); tokens/s = m / mean entry time (the 2x "
+                         "projection overlap of adjacent windows is counted as work)")
         return res
     if name == "hca_prefill":
         wl = W.WORKLOADS[name]
@@ -727,7 +796,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of timed oracle work for the headline's CPU baseline (a third for each secondary)")
     ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192", "indexer_L8192",
-                                                              "csa_decode", "hybrid_decode"],
+                                                              "csa_decode", "hybrid_decode", "front_end_L16384"],
                     help="run one small kernel case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:
@@ -750,7 +819,7 @@ def main():
     head = measure(args.workload, C, args, world, rank, local, peaks, flush)
     secondary = {}
     if args.secondary == "all" and args.workload == "csa_prefill":
-        for name in ("hca_prefill", "csa_decode", "hybrid_decode"):
+        for name in ("hca_prefill", "front_end_prefill", "csa_decode", "hybrid_decode"):
             r = measure(name, C, args, world, rank, local, peaks, flush, with_e2e=False, min_timed_ms=500.0)
             secondary[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "kernel_ms", "roofline",
                                                   "clocks", "config", "steps")}

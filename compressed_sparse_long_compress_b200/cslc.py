@@ -28,6 +28,7 @@ ABI_SYMBOLS = [
     "csa_indexer_topk_workspace_bytes", "csa_indexer_topk", "csa_topk", "csa_sparse_attn",
     "hca_dense_attn", "cslc_quantize_kv_mixed", "cslc_decode_workspace_bytes", "cslc_decode_step",
     "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc", "cslc_decode_append",
+    "csa_compress_front_end", "hca_compress_front_end",
 ]
 
 
@@ -72,6 +73,8 @@ def _load():
         "cslc_decode_topk": (c_int, [P, P, c_int, c_int, c_int, P, P, c_size_t, P]),
         "cslc_decode_topk_noalloc": (c_int, [P, P, c_int, c_int, c_int, P, P]),
         "cslc_decode_append": (c_int, [P, P, P, P, P, P, P, c_int, c_int, c_int, P, P, P, P, P, P, P, P, c_int, P, P]),
+        "csa_compress_front_end": (c_int, [P, P, P, c_int, c_int, c_int, c_int, P, P]),
+        "hca_compress_front_end": (c_int, [P, P, P, c_int, c_int, c_int, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -145,6 +148,20 @@ def hca_compress(c, z, pos_bias, m_prime: int = 128, out=None, stream=None):
         out = torch.empty(B, L // m_prime, D, dtype=BF16, device=c.device)
     _need(out, BF16, "out", (B, L // m_prime, D))
     _check(LIB.hca_compress(_ptr(c), _ptr(z), _ptr(pos_bias), B, L, D, m_prime, _ptr(out), _stream(stream)))
+    return out
+
+
+def compress_front_end(h, W, pos_bias, m: int, overlap: bool, out=None, stream=None):
+    """Entries from hidden states h [B, L, d_model]: W [4, 128, d_model] (CSA)
+    or [2, 128, d_model] (HCA, m = 128); see csa_compress_front_end."""
+    B, L, dm = h.shape
+    _need(h, BF16, "h"); _need(W, BF16, "W", (4 if overlap else 2, 128, dm))
+    _need(pos_bias, BF16, "pos_bias", (2 * m if overlap else m, 128))
+    if out is None:
+        out = torch.empty(B, L // m, 128, dtype=BF16, device=h.device)
+    _need(out, BF16, "out", (B, L // m, 128))
+    fn = LIB.csa_compress_front_end if overlap else LIB.hca_compress_front_end
+    _check(fn(_ptr(h), _ptr(W), _ptr(pos_bias), B, L, dm, m, _ptr(out), _stream(stream)))
     return out
 
 

@@ -43,6 +43,9 @@ size_t decode_workspace_bytes(const cslc_decode_layer*, int, int, int);
 int sparse_attn_sm100_read_error();
 int dense_attn_sm100_read_error();
 int indexer_sm100_read_error();
+int front_end_sm100_read_error();
+cslc_status launch_front_end(const uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int, int, uint16_t*,
+                             cudaStream_t);
 size_t decode_topk_workspace_bytes(int, int, int);
 cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*, size_t, cudaStream_t);
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
@@ -128,6 +131,9 @@ cslc_status cslc_sync_status(cslc_stream_t stream) {
   const int code3 = indexer_sm100_read_error();
   if (code3 != 0)
     return set_error(CSLC_ERR_DEVICE_CHECK, "csa_indexer_topk: a pipeline wait timed out (code %d)", code3);
+  const int code4 = front_end_sm100_read_error();
+  if (code4 != 0)
+    return set_error(CSLC_ERR_DEVICE_CHECK, "compressor front end: a pipeline wait timed out (code %d)", code4);
   return CSLC_OK;
 }
 
@@ -153,6 +159,34 @@ cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z, const cslc_bf16
   if ((long long)B * (L / m_prime) == 0) return CSLC_OK;
   REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(pos_bias); REQUIRE_PTR(out);
   return launch_compress(c, z, nullptr, nullptr, pos_bias, B, L, D, m_prime, 0, out, stream);
+}
+
+static cslc_status front_end_common(const char* fn, const cslc_bf16* h, const cslc_bf16* W,
+                                    const cslc_bf16* pos_bias, int B, int L, int d_model, cslc_bf16* out) {
+  REQUIRE(B >= 0 && L >= 0 && d_model >= 0, CSLC_ERR_SHAPE, "%s: negative size", fn);
+  REQUIRE(d_model >= 64 && d_model % 64 == 0 && d_model <= 65536, CSLC_ERR_UNSUPPORTED,
+          "%s: d_model must be a multiple of 64 in [64, 65536]", fn);
+  REQUIRE((long long)B * L < (1ll << 31), CSLC_ERR_UNSUPPORTED, "%s: B * L must be below 2^31", fn);
+  REQUIRE_PTR(h); REQUIRE_PTR(W); REQUIRE_PTR(pos_bias); REQUIRE_PTR(out);
+  return CSLC_OK;
+}
+
+cslc_status csa_compress_front_end(const cslc_bf16* h, const cslc_bf16* W, const cslc_bf16* pos_bias, int B, int L,
+                                   int d_model, int m, cslc_bf16* out, cslc_stream_t stream) {
+  REQUIRE(is_pow2(m) && m <= 64, CSLC_ERR_UNSUPPORTED, "csa_compress_front_end: m must be a power of two <= 64");
+  if (B >= 0 && L >= 0 && (long long)B * (L / m) == 0) return CSLC_OK;
+  const cslc_status st = front_end_common("csa_compress_front_end", h, W, pos_bias, B, L, d_model, out);
+  if (st != CSLC_OK) return st;
+  return launch_front_end(h, W, pos_bias, B, L, d_model, m, 1, out, stream);
+}
+
+cslc_status hca_compress_front_end(const cslc_bf16* h, const cslc_bf16* W, const cslc_bf16* pos_bias, int B, int L,
+                                   int d_model, int m_prime, cslc_bf16* out, cslc_stream_t stream) {
+  REQUIRE(m_prime == 128, CSLC_ERR_UNSUPPORTED, "hca_compress_front_end: m' must be 128");
+  if (B >= 0 && L >= 0 && (long long)B * (L / m_prime) == 0) return CSLC_OK;
+  const cslc_status st = front_end_common("hca_compress_front_end", h, W, pos_bias, B, L, d_model, out);
+  if (st != CSLC_OK) return st;
+  return launch_front_end(h, W, pos_bias, B, L, d_model, m_prime, 0, out, stream);
 }
 
 size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {

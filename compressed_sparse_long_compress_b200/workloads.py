@@ -62,6 +62,25 @@ class DecodeShape:
 
 
 @dataclass(frozen=True)
+class FrontEndShape:
+    """Compressor front end: hidden states [B, L, d_model] through the learned
+    projections into compressed entries (window ratio m, overlap = CSA)."""
+    B: int
+    L: int
+    d_model: int
+    m: int = 4
+    overlap: bool = True
+
+    @property
+    def n_c(self) -> int:
+        return self.L // self.m
+
+    @property
+    def n_proj(self) -> int:
+        return 4 if self.overlap else 2
+
+
+@dataclass(frozen=True)
 class Workload:
     wid: int
     name: str
@@ -70,6 +89,7 @@ class Workload:
     hca: PrefillShape | None = None
     decode: DecodeShape | None = None
     extra: dict = field(default_factory=dict)
+    front_end: FrontEndShape | None = None
 
 
 WORKLOADS = {
@@ -103,6 +123,12 @@ WORKLOADS = {
         "CSA 262144 entries (top-k 1024), HCA 8192 entries; 64 heads x 128, mixed KV",
         decode=DecodeShape(B=8, H=64, kinds=("csa", "hca", "csa", "hca"),
                            n_entries=(262144, 8192, 262144, 8192)),
+    ),
+    "front_end_prefill": Workload(
+        6, "front_end_prefill",
+        "CSA compressor front end, batch 1, L=65536 hidden states of d_model=7168 -> 4 learned projections "
+        "(4 x 128) -> overlapped 2m-window compression, m=4 -> 16384 entries",
+        front_end=FrontEndShape(B=1, L=65536, d_model=7168, m=4, overlap=True),
     ),
 }
 
@@ -161,6 +187,19 @@ def prefill_inputs(s: PrefillShape, wid: int, device="cpu", with_indexer=None,
         out["w"] = rand_bf16((B, L, s.HI), seed_of(wid, T_W), device)
         out["k_idx"] = randn_bf16((B, s.n_c, s.dI), seed_of(wid, T_KIDX), device)
     return out
+
+
+T_H, T_W = 14, 15
+
+
+def front_end_inputs(s: FrontEndShape, wid: int, device="cpu"):
+    """Hidden states h ~ N(0, 1), projection weights ~ N(0, 1/d_model) (so the
+    projections are ~ N(0, 1)) and positional bias ~ N(0, 0.1^2), all bf16."""
+    return {
+        "h": randn_bf16((s.B, s.L, s.d_model), seed_of(wid, T_H), device),
+        "W": randn_bf16((s.n_proj, 128, s.d_model), seed_of(wid, T_W), device, std=s.d_model ** -0.5),
+        "pos_bias": randn_bf16((2 * s.m if s.overlap else s.m, 128), seed_of(wid, T_BIAS), device, std=0.1),
+    }
 
 
 def decode_layer_inputs(d: DecodeShape, layer: int, wid: int, device="cpu", n_max=None):

@@ -107,6 +107,30 @@ cslc_status hca_compress(const cslc_bf16* c, const cslc_bf16* z,
                          const cslc_bf16* pos_bias, int B, int L, int D,
                          int m_prime, cslc_bf16* out, cslc_stream_t stream);
 
+/* Compressor front end ("读完这篇…" §三 压缩机制: 4 learnable W matrices and 2
+ * learnable B matrices): the compressed entries straight from the hidden
+ * states, the projections and the window compression in one pass.
+ *
+ * CSA: W [4, 128, d_model] bf16 holds W^{a,KV}, W^{b,KV}, W^{a,Z}, W^{b,Z},
+ * each in [output, input] layout: per token t, c^a_t = W^{a,KV} h_t,
+ * c^b_t = W^{b,KV} h_t, z^a_t = W^{a,Z} h_t, z^b_t = W^{b,Z} h_t (fp32
+ * accumulation of bf16 products, not rounded); entry i is csa_compress's
+ * window softmax with the C^a half reading (c^a, z^a) and the C^b half
+ * (c^b, z^b): pos_bias [2m, 128] bf16 holds B^b (slots 0..m-1) then B^a.
+ *   h [B, L, d_model] bf16; out [B, floor(L/m), 128] bf16.
+ * Requires d_model a multiple of 64 (<= 65536), m a power of two <= 64,
+ * B * L < 2^31. One launch; no workspace.
+ *
+ * HCA: W [2, 128, d_model] (W^{KV}, W^{Z}), pos_bias [m', 128], m' = 128;
+ * entry i compresses tokens im' .. im'+m'-1 with c = W^{KV} h, z = W^{Z} h.
+ */
+cslc_status csa_compress_front_end(const cslc_bf16* h, const cslc_bf16* W, const cslc_bf16* pos_bias,
+                                   int B, int L, int d_model, int m, cslc_bf16* out,
+                                   cslc_stream_t stream);
+cslc_status hca_compress_front_end(const cslc_bf16* h, const cslc_bf16* W, const cslc_bf16* pos_bias,
+                                   int B, int L, int d_model, int m_prime, cslc_bf16* out,
+                                   cslc_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Lightning indexer + top-k ("读完这篇…" §三 闪电索引; first page §1.1 top-k=1024)
  *
