@@ -29,6 +29,7 @@ ABI_SYMBOLS = [
     "hca_dense_attn", "cslc_quantize_kv_mixed", "cslc_decode_workspace_bytes", "cslc_decode_step",
     "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc", "cslc_decode_append",
     "csa_compress_front_end", "hca_compress_front_end",
+    "csa_indexer_topk_bf16_workspace_bytes", "csa_indexer_topk_bf16", "csa_topk_bf16",
 ]
 
 
@@ -74,6 +75,10 @@ def _load():
         "cslc_decode_topk_noalloc": (c_int, [P, P, c_int, c_int, c_int, P, P]),
         "cslc_decode_append": (c_int, [P, P, P, P, P, P, P, c_int, c_int, c_int, P, P, P, P, P, P, P, P, c_int, P, P]),
         "csa_compress_front_end": (c_int, [P, P, P, c_int, c_int, c_int, c_int, P, P]),
+        "csa_indexer_topk_bf16_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+        "csa_indexer_topk_bf16": (c_int, [P, P, P, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                          P, P, P, c_size_t, P]),
+        "csa_topk_bf16": (c_int, [P, c_int, c_int, c_int, c_int, c_int, c_int, P, P]),
         "hca_compress_front_end": (c_int, [P, P, P, c_int, c_int, c_int, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -192,6 +197,43 @@ def csa_indexer_topk(q_idx, w, k_idx, m: int, topk: int, q_pos0: int = 0, scores
 
 def indexer_topk_workspace_bytes(B, L, Nc, HI, topk, scores_given=False) -> int:
     return LIB.csa_indexer_topk_workspace_bytes(B, L, Nc, HI, topk, int(scores_given))
+
+
+def csa_indexer_topk_bf16(q_idx, w, k_idx, m: int, topk: int, q_pos0: int = 0, scores=None, idx=None,
+                          ws=None, stream=None):
+    """As csa_indexer_topk with bf16-stored scores (scores=True allocates a
+    [B, L, Nc] bf16 tensor)."""
+    B, L, HI, dI = q_idx.shape
+    Nc = k_idx.shape[1]
+    _need(q_idx, BF16, "q_idx"); _need(w, BF16, "w", (B, L, HI)); _need(k_idx, BF16, "k_idx", (B, Nc, dI))
+    if scores is True:
+        scores = torch.empty(B, L, Nc, dtype=BF16, device=q_idx.device)
+    if scores is not None:
+        _need(scores, BF16, "scores", (B, L, Nc))
+    if idx is None:
+        idx = torch.empty(B, L, topk, dtype=I32, device=q_idx.device)
+    _need(idx, I32, "idx", (B, L, topk))
+    nbytes = LIB.csa_indexer_topk_bf16_workspace_bytes(B, L, Nc, HI, topk, int(scores is not None))
+    if nbytes and (ws is None or ws.numel() < nbytes):
+        ws = torch.empty(nbytes, dtype=U8, device=q_idx.device)
+    _check(LIB.csa_indexer_topk_bf16(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, L, Nc, HI, dI, m, q_pos0, topk,
+                                     _ptr(scores), _ptr(idx), _ptr(ws) if nbytes else None,
+                                     ws.numel() if (nbytes and ws is not None) else 0, _stream(stream)))
+    return idx, scores
+
+
+def indexer_topk_bf16_workspace_bytes(B, L, Nc, HI, topk, scores_given=False) -> int:
+    return LIB.csa_indexer_topk_bf16_workspace_bytes(B, L, Nc, HI, topk, int(scores_given))
+
+
+def csa_topk_bf16(scores, m: int, topk: int, q_pos0: int = 0, idx=None, stream=None):
+    B, L, Nc = scores.shape
+    _need(scores, BF16, "scores")
+    if idx is None:
+        idx = torch.empty(B, L, topk, dtype=I32, device=scores.device)
+    _need(idx, I32, "idx", (B, L, topk))
+    _check(LIB.csa_topk_bf16(_ptr(scores), B, L, Nc, m, q_pos0, topk, _ptr(idx), _stream(stream)))
+    return idx
 
 
 def csa_topk(scores, m: int, topk: int, q_pos0: int = 0, idx=None, stream=None):

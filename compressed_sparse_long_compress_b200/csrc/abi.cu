@@ -32,8 +32,8 @@ cslc_status launch_decode_append(const uint16_t*, const uint16_t*, const uint16_
                                  uint16_t*, uint8_t*, uint16_t*, float*, uint16_t*, int, int32_t*, cudaStream_t);
 cslc_status launch_quantize_kv(const uint16_t*, long long, uint8_t*, uint16_t*, float*, cudaStream_t);
 cslc_status launch_indexer_scores(const uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int,
-                                  int, int, int, int, float*, int, cudaStream_t);
-cslc_status launch_topk_rows(const float*, int, int, int, int, int, int, int, int, int, int32_t*,
+                                  int, int, int, int, void*, bool, int, cudaStream_t);
+cslc_status launch_topk_rows(const void*, bool, int, int, int, int, int, int, int, int, int, int32_t*,
                              cudaStream_t);
 cslc_status launch_sparse_attn(const uint16_t*, const uint16_t*, const int32_t*, int, int, int, int, int,
                                float, uint16_t*, float*, cudaStream_t);
@@ -51,7 +51,7 @@ cslc_status run_decode_step(const cslc_decode_layer*, int, int, int, int, void*,
 cslc_status run_decode_topk(const float*, const int32_t*, int, int, int, int32_t*, void*, cudaStream_t);
 
 constexpr int kMaxTopk = 2048;
-constexpr int kMaxPrefillTopkNc = 45056;   // a row of scores must fit in shared memory
+constexpr int kMaxPrefillTopkNc = 786432;   // a row's selection masks (Nc / 4 bytes) fit in shared memory
 
 static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -70,9 +70,9 @@ static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 // this many rows, two blocks in flight: the top-k of one block runs on an
 // auxiliary stream beside the indexer of the next, so neither launch's tail
 // leaves SMs idle.
-static int score_block_rows(int Nc) {
+static int score_block_rows(int Nc, int score_bytes = 4) {
   const long long budget = 512ll << 20;   // bytes of scores per block
-  long long rows = budget / ((long long)Nc * 4);
+  long long rows = budget / ((long long)Nc * score_bytes);
   rows = rows < 64 ? 64 : rows;
   rows = (rows / 64) * 64;
   return (int)rows;
@@ -189,86 +189,122 @@ cslc_status hca_compress_front_end(const cslc_bf16* h, const cslc_bf16* W, const
   return launch_front_end(h, W, pos_bias, B, L, d_model, m_prime, 0, out, stream);
 }
 
-size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {
-  (void)HI; (void)topk;
+static size_t indexer_ws_bytes(int B, int L, int Nc, int score_bytes, int scores_given) {
   if (scores_given || B <= 0 || L <= 0 || Nc <= 0) return 0;
-  const int rows = score_block_rows(Nc);
+  const int rows = score_block_rows(Nc, score_bytes);
   const int R = L < rows ? L : rows;
   const int n_buf = L > R ? 2 : 1;
-  return (size_t)n_buf * B * R * Nc * 4;
+  return (size_t)n_buf * B * R * Nc * score_bytes;
+}
+
+// The indexer and the top-k, with fp32 or bf16 scores (bf16: each fp32 score
+// rounded to nearest even before it is stored and selected on).
+static cslc_status indexer_topk_impl(const char* fn, const cslc_bf16* q_idx, const cslc_bf16* w,
+                                     const cslc_bf16* k_idx, int B, int L, int Nc, int HI, int dI, int m,
+                                     int q_pos0, int topk, void* scores, bool bf16, int32_t* idx, void* ws,
+                                     size_t ws_bytes, cudaStream_t stream) {
+  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE, "%s: negative size / m < 1", fn);
+  REQUIRE(dI == kDI, CSLC_ERR_UNSUPPORTED, "%s: d_I must be 64 (got %d)", fn, dI);
+  REQUIRE(HI >= 1 && HI <= 16, CSLC_ERR_UNSUPPORTED, "%s: H_I must be in [1, 16]", fn);
+  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "%s: topk must be in [1, 2048]", fn);
+  REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "%s: Nc must be <= %d", fn, kMaxPrefillTopkNc);
+  if ((long long)B * L == 0) return CSLC_OK;
+  REQUIRE_PTR(idx);
+  if (Nc > 0) { REQUIRE_PTR(q_idx); REQUIRE_PTR(w); REQUIRE_PTR(k_idx); }
+  if (scores) REQUIRE_PTR(scores);
+  const int sb = bf16 ? 2 : 4;
+  const size_t need = indexer_ws_bytes(B, L, Nc, sb, scores != nullptr);
+  if (need) {
+    REQUIRE(ws != nullptr && ws_bytes >= need, CSLC_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", fn, need);
+    REQUIRE(aligned16(ws), CSLC_ERR_ALIGN, "%s: ws is not 16-byte aligned", fn);
+  }
+  cslc_status st;
+  if (scores) {
+    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, scores, bf16, L, stream);
+    if (st != CSLC_OK) return st;
+    return launch_topk_rows(scores, bf16, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
+  }
+  const int rows = score_block_rows(Nc, sb);
+  const int R = L < rows ? L : rows;
+  uint8_t* buf = static_cast<uint8_t*>(ws);
+  if (L <= R || Nc == 0) {
+    if (Nc > 0) {
+      st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, buf, bf16, R, stream);
+      if (st != CSLC_OK) return st;
+    }
+    return launch_topk_rows(buf, bf16, R, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
+  }
+  BlockOverlap* o = nullptr;
+  st = block_overlap(&o);
+  if (st != CSLC_OK) return st;
+  const size_t block_bytes = (size_t)B * R * Nc * sb;
+  int last = 0;
+  for (int i = 0, r0 = 0; r0 < L; ++i, r0 += R) {
+    const int r1 = r0 + R < L ? r0 + R : L;
+    const int j = i & 1;
+    uint8_t* bj = buf + j * block_bytes;
+    cudaError_t e = i >= 2 ? cudaStreamWaitEvent(stream, o->freed[j], 0) : cudaSuccess;
+    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, r0, r1, bj, bf16, R, stream);
+    if (st != CSLC_OK) return st;
+    e = cudaEventRecord(o->ready[j], stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(o->aux, o->ready[j], 0);
+    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+    st = launch_topk_rows(bj, bf16, R, r0, r1, B, L, Nc, m, q_pos0, topk, idx, o->aux);
+    if (st != CSLC_OK) return st;
+    e = cudaEventRecord(o->freed[j], o->aux);
+    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+    last = j;
+  }
+  // join: `stream` continues after the last top-k (the auxiliary stream runs in order)
+  const cudaError_t e = cudaStreamWaitEvent(stream, o->freed[last], 0);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  return CSLC_OK;
+}
+
+static cslc_status topk_impl(const char* fn, const void* scores, bool bf16, int B, int L, int Nc, int m, int q_pos0,
+                             int topk, int32_t* idx, cudaStream_t stream) {
+  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE, "%s: bad size", fn);
+  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "%s: topk must be in [1, 2048]", fn);
+  REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "%s: Nc must be <= %d", fn, kMaxPrefillTopkNc);
+  if ((long long)B * L == 0) return CSLC_OK;
+  REQUIRE_PTR(idx);
+  if (Nc > 0) REQUIRE_PTR(scores);
+  return launch_topk_rows(scores, bf16, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
+}
+
+size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {
+  (void)HI; (void)topk;
+  return indexer_ws_bytes(B, L, Nc, 4, scores_given);
 }
 
 cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w, const cslc_bf16* k_idx, int B,
                              int L, int Nc, int HI, int dI, int m, int q_pos0, int topk, float* scores,
                              int32_t* idx, void* ws, size_t ws_bytes, cslc_stream_t stream) {
-  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE,
-          "csa_indexer_topk: negative size / m < 1");
-  REQUIRE(dI == kDI, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: d_I must be 64 (got %d)", dI);
-  REQUIRE(HI >= 1 && HI <= 16, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: H_I must be in [1, 16]");
-  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: topk must be in [1, 2048]");
-  REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "csa_indexer_topk: Nc must be <= %d", kMaxPrefillTopkNc);
-  if ((long long)B * L == 0) return CSLC_OK;
-  REQUIRE_PTR(idx);
-  if (Nc > 0) { REQUIRE_PTR(q_idx); REQUIRE_PTR(w); REQUIRE_PTR(k_idx); }
-  if (scores) REQUIRE_PTR(scores);
-  const size_t need = csa_indexer_topk_workspace_bytes(B, L, Nc, HI, topk, scores != nullptr);
-  if (need) {
-    REQUIRE(ws != nullptr && ws_bytes >= need, CSLC_ERR_WORKSPACE,
-            "csa_indexer_topk: workspace of %zu bytes needed", need);
-    REQUIRE(aligned16(ws), CSLC_ERR_ALIGN, "csa_indexer_topk: ws is not 16-byte aligned");
-  }
-  cslc_status st;
-  if (scores) {
-    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, scores, L, stream);
-    if (st != CSLC_OK) return st;
-    return launch_topk_rows(scores, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
-  }
-  const int R = L < score_block_rows(Nc) ? L : score_block_rows(Nc);
-  float* buf = static_cast<float*>(ws);
-  if (L <= R || Nc == 0) {
-    if (Nc > 0) {
-      st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, buf, R, stream);
-      if (st != CSLC_OK) return st;
-    }
-    return launch_topk_rows(buf, R, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
-  }
-  BlockOverlap* o = nullptr;
-  st = block_overlap(&o);
-  if (st != CSLC_OK) return st;
-  const size_t block_floats = (size_t)B * R * Nc;
-  int last = 0;
-  for (int i = 0, r0 = 0; r0 < L; ++i, r0 += R) {
-    const int r1 = r0 + R < L ? r0 + R : L;
-    const int j = i & 1;
-    float* bj = buf + j * block_floats;
-    cudaError_t e = i >= 2 ? cudaStreamWaitEvent(stream, o->freed[j], 0) : cudaSuccess;
-    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
-    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, r0, r1, bj, R, stream);
-    if (st != CSLC_OK) return st;
-    e = cudaEventRecord(o->ready[j], stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(o->aux, o->ready[j], 0);
-    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
-    st = launch_topk_rows(bj, R, r0, r1, B, L, Nc, m, q_pos0, topk, idx, o->aux);
-    if (st != CSLC_OK) return st;
-    e = cudaEventRecord(o->freed[j], o->aux);
-    if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
-    last = j;
-  }
-  // join: `stream` continues after the last top-k (the auxiliary stream runs in order)
-  const cudaError_t e = cudaStreamWaitEvent(stream, o->freed[last], 0);
-  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: %s", cudaGetErrorString(e));
-  return CSLC_OK;
+  return indexer_topk_impl("csa_indexer_topk", q_idx, w, k_idx, B, L, Nc, HI, dI, m, q_pos0, topk, scores, false,
+                           idx, ws, ws_bytes, stream);
+}
+
+size_t csa_indexer_topk_bf16_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {
+  (void)HI; (void)topk;
+  return indexer_ws_bytes(B, L, Nc, 2, scores_given);
+}
+
+cslc_status csa_indexer_topk_bf16(const cslc_bf16* q_idx, const cslc_bf16* w, const cslc_bf16* k_idx, int B,
+                                  int L, int Nc, int HI, int dI, int m, int q_pos0, int topk, cslc_bf16* scores,
+                                  int32_t* idx, void* ws, size_t ws_bytes, cslc_stream_t stream) {
+  return indexer_topk_impl("csa_indexer_topk_bf16", q_idx, w, k_idx, B, L, Nc, HI, dI, m, q_pos0, topk, scores,
+                           true, idx, ws, ws_bytes, stream);
 }
 
 cslc_status csa_topk(const float* scores, int B, int L, int Nc, int m, int q_pos0, int topk, int32_t* idx,
                      cslc_stream_t stream) {
-  REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE, "csa_topk: bad size");
-  REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "csa_topk: topk must be in [1, 2048]");
-  REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "csa_topk: Nc must be <= %d", kMaxPrefillTopkNc);
-  if ((long long)B * L == 0) return CSLC_OK;
-  REQUIRE_PTR(idx);
-  if (Nc > 0) REQUIRE_PTR(scores);
-  return launch_topk_rows(scores, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
+  return topk_impl("csa_topk", scores, false, B, L, Nc, m, q_pos0, topk, idx, stream);
+}
+
+cslc_status csa_topk_bf16(const cslc_bf16* scores, int B, int L, int Nc, int m, int q_pos0, int topk, int32_t* idx,
+                          cslc_stream_t stream) {
+  return topk_impl("csa_topk_bf16", scores, true, B, L, Nc, m, q_pos0, topk, idx, stream);
 }
 
 cslc_status csa_sparse_attn(const cslc_bf16* q, const cslc_bf16* kv, const int32_t* idx, int B, int L, int H,

@@ -22,10 +22,19 @@ constexpr int IDX_TILE = 64;     // entries per key tile
 constexpr int IDX_THREADS = 128;
 constexpr int IDX_SPLIT_TILES = 16;   // key tiles (1024 entries) per CTA
 
+// Score stores: fp32, or bf16 (round to nearest even) for the half-size score path.
+__device__ __forceinline__ void put1(float* p, float v) { *p = v; }
+__device__ __forceinline__ void put1(uint16_t* p, float v) { *p = __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+__device__ __forceinline__ void put2(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+__device__ __forceinline__ void put2(uint16_t* p, float a, float b) {
+  *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+}
+
+template <typename OutT>
 __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
     const uint16_t* __restrict__ q_idx, const uint16_t* __restrict__ w,
     const uint16_t* __restrict__ k_idx, int L, int Nc, int HI, int m, int q_pos0,
-    int row_begin, int row_end, float* __restrict__ scores, int rows_in_buf) {
+    int row_begin, int row_end, OutT* __restrict__ scores, int rows_in_buf) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* q_s = smem;                                        // [HI][64 rows][128 B]
   uint8_t* k_s = smem + HI * IDX_ROWS * 128;                  // [2][64 entries][128 B]
@@ -134,27 +143,25 @@ __global__ void __launch_bounds__(IDX_THREADS, 2) indexer_scores_kernel(
       // store: entries past n_vis inside this tile get -inf; never past Nc. Pairs
       // go out as one 8-byte store only when every row starts 8-byte aligned.
       const bool pair_ok = (Nc & 1) == 0;
-      float* sa = scores + ((size_t)b * rows_in_buf + (ra - row_begin)) * (size_t)Nc;
-      float* sb = scores + ((size_t)b * rows_in_buf + (rb - row_begin)) * (size_t)Nc;
+      OutT* sa = scores + ((size_t)b * rows_in_buf + (ra - row_begin)) * (size_t)Nc;
+      OutT* sb = scores + ((size_t)b * rows_in_buf + (rb - row_begin)) * (size_t)Nc;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int col = e0 + nt * 8 + 2 * tq;
         if (ra < row_end && e0 < nva) {
           if (pair_ok && col + 1 < Nc) {
-            float2 v = make_float2(col < nva ? acc[nt][0] : -INFINITY, col + 1 < nva ? acc[nt][1] : -INFINITY);
-            *reinterpret_cast<float2*>(sa + col) = v;
+            put2(sa + col, col < nva ? acc[nt][0] : -INFINITY, col + 1 < nva ? acc[nt][1] : -INFINITY);
           } else {
-            if (col < Nc) sa[col] = col < nva ? acc[nt][0] : -INFINITY;
-            if (col + 1 < Nc) sa[col + 1] = col + 1 < nva ? acc[nt][1] : -INFINITY;
+            if (col < Nc) put1(sa + col, col < nva ? acc[nt][0] : -INFINITY);
+            if (col + 1 < Nc) put1(sa + col + 1, col + 1 < nva ? acc[nt][1] : -INFINITY);
           }
         }
         if (rb < row_end && e0 < nvb) {
           if (pair_ok && col + 1 < Nc) {
-            float2 v = make_float2(col < nvb ? acc[nt][2] : -INFINITY, col + 1 < nvb ? acc[nt][3] : -INFINITY);
-            *reinterpret_cast<float2*>(sb + col) = v;
+            put2(sb + col, col < nvb ? acc[nt][2] : -INFINITY, col + 1 < nvb ? acc[nt][3] : -INFINITY);
           } else {
-            if (col < Nc) sb[col] = col < nvb ? acc[nt][2] : -INFINITY;
-            if (col + 1 < Nc) sb[col + 1] = col + 1 < nvb ? acc[nt][3] : -INFINITY;
+            if (col < Nc) put1(sb + col, col < nvb ? acc[nt][2] : -INFINITY);
+            if (col + 1 < Nc) put1(sb + col + 1, col + 1 < nvb ? acc[nt][3] : -INFINITY);
           }
         }
       }
@@ -171,23 +178,26 @@ size_t indexer_smem_bytes(int HI) {
 bool indexer_sm100_supported(int HI);
 cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int B,
                                  int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
-                                 float* scores, int rows_in_buf, cudaStream_t stream);
+                                 void* scores, bool bf16_out, int rows_in_buf, cudaStream_t stream);
 
+// scores: fp32 [rows][Nc], or bf16 when bf16_out
 cslc_status launch_indexer_scores(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
                                   int B, int L, int Nc, int HI, int m, int q_pos0, int row_begin,
-                                  int row_end, float* scores, int rows_in_buf, cudaStream_t stream) {
+                                  int row_end, void* scores, bool bf16_out, int rows_in_buf, cudaStream_t stream) {
   if (row_end <= row_begin || B == 0) return CSLC_OK;
   // tensor-core path when whole TMA boxes fit the operands (256 query pairs,
   // 128 entries); the mma.sync kernel below takes the rest
   if (indexer_sm100_supported(HI) && (long long)B * L * HI >= 256 && (long long)B * Nc >= 128)
-    return launch_indexer_sm100(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores,
+    return launch_indexer_sm100(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, bf16_out,
                                 rows_in_buf, stream);
   const size_t smem = indexer_smem_bytes(HI);
   static int configured_for = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_for != dev) {
-    cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(indexer_scores_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)indexer_smem_bytes(16));
+    cudaFuncSetAttribute(indexer_scores_kernel<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)indexer_smem_bytes(16));
     configured_for = dev;
   }
@@ -196,8 +206,12 @@ cslc_status launch_indexer_scores(const uint16_t* q_idx, const uint16_t* w, cons
   const int n_split = ((nv_max + IDX_TILE - 1) / IDX_TILE + IDX_SPLIT_TILES - 1) / IDX_SPLIT_TILES;
   if (n_split == 0) return CSLC_OK;
   dim3 grid(n_rb * n_split, B);
-  indexer_scores_kernel<<<grid, IDX_THREADS, smem, stream>>>(q_idx, w, k_idx, L, Nc, HI, m, q_pos0,
-                                                             row_begin, row_end, scores, rows_in_buf);
+  if (bf16_out)
+    indexer_scores_kernel<uint16_t><<<grid, IDX_THREADS, smem, stream>>>(
+        q_idx, w, k_idx, L, Nc, HI, m, q_pos0, row_begin, row_end, static_cast<uint16_t*>(scores), rows_in_buf);
+  else
+    indexer_scores_kernel<float><<<grid, IDX_THREADS, smem, stream>>>(
+        q_idx, w, k_idx, L, Nc, HI, m, q_pos0, row_begin, row_end, static_cast<float*>(scores), rows_in_buf);
   return check_launch("indexer_scores_kernel");
 }
 

@@ -73,10 +73,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 }  // namespace
 
-template <int HI>
+// Score store: fp32, or bf16 (round to nearest even) for the half-size score path.
+__device__ __forceinline__ void store_score(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_score(uint16_t* p, float v) { *p = __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+template <int HI, typename OutT>
 __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
     const uint16_t* __restrict__ w, int B, int L, int Nc, int m, int q_pos0, int row_begin, int row_end,
-    float* __restrict__ scores, int rows_in_buf, const __grid_constant__ CUtensorMap tm_q,
+    OutT* __restrict__ scores, int rows_in_buf, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_k) {
   constexpr int RT = IX_NP / HI;                 // query rows per tile
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       const float4* wr = reinterpret_cast<const float4*>(w_s + qs * IX_NP + part * IX_EPI_COLS);
       const int* nvr = nv_s + qs * IX_NP + part * RH;
       const int r0 = t0 + part * RH;                  // first row of this warp's part
-      float* out0 = scores + ((size_t)b * rows_in_buf + (r0 - row_begin)) * (size_t)Nc;
+      OutT* out0 = scores + ((size_t)b * rows_in_buf + (r0 - row_begin)) * (size_t)Nc;
       for (int et = et0; et < et0 + n_et; ++et, ++kt) {
         const int ds = kt & 1;
         bool d_ok = true;
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
                 if (q & 1) s1 = fmaf(wq[q], x, s1); else s0 = fmaf(wq[q], x, s0);
               }
             }
-            if (e < nvr[r]) out0[(size_t)r * Nc + e] = s0 + s1;
+            if (e < nvr[r]) store_score(out0 + (size_t)r * Nc + e, s0 + s1);
           }
         }
         tc_fence_before();
@@ -294,9 +298,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
 
 bool indexer_sm100_supported(int HI) { return HI == 1 || HI == 2 || HI == 4 || HI == 8 || HI == 16; }
 
-cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int B,
-                                 int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
-                                 float* scores, int rows_in_buf, cudaStream_t stream) {
+template <typename OutT>
+static cslc_status launch_indexer_sm100_t(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int B,
+                                          int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
+                                          OutT* scores, int rows_in_buf, cudaStream_t stream) {
   static int configured_for = -1;
   static int n_sm = 148;
   int dev = 0;
@@ -304,11 +309,11 @@ cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const
   const size_t smem = 1024 + 2 * IX_Q_BYTES + IX_KSTAGES * IX_K_BYTES + 2 * IX_NP * (sizeof(float) + sizeof(int)) +
                       sizeof(IxSmall);
   if (configured_for != dev) {
-    cudaFuncSetAttribute(indexer_sm100_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<1, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<2, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<4, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<8, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<16, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     configured_for = dev;
   }
@@ -322,13 +327,24 @@ cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const
       !make_tmap_bf16_2d(&tm_k, k_idx, (uint64_t)B * Nc, kDI, kDI * 2, IX_ET, 64))
     return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: tensor map encoding failed");
   switch (HI) {
-    case 1: indexer_sm100_kernel<1><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 2: indexer_sm100_kernel<2><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 4: indexer_sm100_kernel<4><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 8: indexer_sm100_kernel<8><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    default: indexer_sm100_kernel<16><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 1: indexer_sm100_kernel<1, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 2: indexer_sm100_kernel<2, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 4: indexer_sm100_kernel<4, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 8: indexer_sm100_kernel<8, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    default: indexer_sm100_kernel<16, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
   }
   return check_launch("indexer_sm100_kernel");
+}
+
+// scores: fp32 [rows][Nc], or bf16 when bf16_out
+cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int B,
+                                 int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
+                                 void* scores, bool bf16_out, int rows_in_buf, cudaStream_t stream) {
+  if (bf16_out)
+    return launch_indexer_sm100_t(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end,
+                                  static_cast<uint16_t*>(scores), rows_in_buf, stream);
+  return launch_indexer_sm100_t(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end,
+                                static_cast<float*>(scores), rows_in_buf, stream);
 }
 
 int indexer_sm100_read_error() {

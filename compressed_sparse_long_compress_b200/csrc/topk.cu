@@ -201,8 +201,23 @@ __device__ __forceinline__ int tk_block_excl_scan(int v, int* wtot, int& total) 
 // Rows for which a check fails (degenerate sampled range, too many collected
 // keys, bounds that miss the k-th score, e.g. through NaN scores) take the
 // exact 8-bit radix select over order-preserving keys read from the row.
+// Score rows are fp32, or bf16 (the half-size score path; a bf16 score
+// converts to fp32 exactly, so the selection below is the same code).
+__device__ __forceinline__ float score_at(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float score_at(const uint16_t* p) { return bf16_to_f(__ldg(p)); }
+__device__ __forceinline__ float4 score4(const float* p, bool last_use) {
+  const float4* v = reinterpret_cast<const float4*>(p);
+  return last_use ? __ldcs(v) : __ldg(v);
+}
+__device__ __forceinline__ float4 score4(const uint16_t* p, bool last_use) {
+  const uint2* v = reinterpret_cast<const uint2*>(p);
+  const uint2 u = last_use ? __ldcs(v) : __ldg(v);
+  return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+}
+
+template <typename ScoreT>
 __global__ void __launch_bounds__(TOPK_THREADS, 8) topk_rows_kernel(
-    const float* __restrict__ scores, int rows_in_buf, int row_begin, int L, int Nc, int m,
+    const ScoreT* __restrict__ scores, int rows_in_buf, int row_begin, int L, int Nc, int m,
     int q_pos0, int topk, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint32_t nibw[];   // 4-bit masks: entries 16w..16w+15 in word w
   uint8_t* nib = reinterpret_cast<uint8_t*>(nibw);
@@ -224,24 +239,21 @@ __global__ void __launch_bounds__(TOPK_THREADS, 8) topk_rows_kernel(
     for (int j = tid; j < topk; j += TOPK_THREADS) out[j] = j < nv ? j : -1;
     return;
   }
-  const float* srow = scores + ((size_t)b * rows_in_buf + (r - row_begin)) * (size_t)Nc;
+  const ScoreT* srow = scores + ((size_t)b * rows_in_buf + (r - row_begin)) * (size_t)Nc;
   const int n_sl = (nv + TK_SLICE - 1) / TK_SLICE;
 #pragma unroll
   for (int j = 0; j < TK_BINS / (4 * TOPK_THREADS); ++j)
     reinterpret_cast<uint4*>(hist)[j * TOPK_THREADS + tid] = make_uint4(0u, 0u, 0u, 0u);
   if (tid == 0) n_cand = 0;
-  const bool vec = (Nc & 3) == 0;   // rows start 16-byte aligned
+  const bool vec = (Nc & 3) == 0;   // rows start 16-byte (fp32) / 8-byte (bf16) aligned
   auto load4 = [&](int e, bool last_use) -> float4 {   // entries e..e+3, NaN past the row
-    if (vec && e + 4 <= nv) {
-      const float4* p = reinterpret_cast<const float4*>(srow + e);
-      return last_use ? __ldcs(p) : __ldg(p);
-    }
+    if (vec && e + 4 <= nv) return score4(srow + e, last_use);
     const float qnan = __int_as_float(0x7fc00000);
     float4 f;
-    f.x = e + 0 < nv ? __ldg(srow + e + 0) : qnan;
-    f.y = e + 1 < nv ? __ldg(srow + e + 1) : qnan;
-    f.z = e + 2 < nv ? __ldg(srow + e + 2) : qnan;
-    f.w = e + 3 < nv ? __ldg(srow + e + 3) : qnan;
+    f.x = e + 0 < nv ? score_at(srow + e + 0) : qnan;
+    f.y = e + 1 < nv ? score_at(srow + e + 1) : qnan;
+    f.z = e + 2 < nv ? score_at(srow + e + 2) : qnan;
+    f.w = e + 3 < nv ? score_at(srow + e + 3) : qnan;
     return f;
   };
   // A. histogram
@@ -416,21 +428,40 @@ __global__ void __launch_bounds__(TOPK_THREADS, 8) topk_rows_kernel(
   }
   // exact radix select over order-preserving keys read from the row
   __syncthreads();
-  auto key_of = [&](int i) { return float_key(__ldg(srow + i)); };
+  auto key_of = [&](int i) { return float_key(score_at(srow + i)); };
   const RadixResult rr = radix_select(key_of, nv, topk, hist, bcast);
   emit_selection(key_of, nv, rr, out, topk, wsum);
 }
 
-cslc_status launch_topk_rows(const float* scores, int rows_in_buf, int row_begin, int row_end,
+// Largest row (entries) the top-k takes: its 4-bit selection masks (Nc / 4
+// bytes of dynamic shared memory) beside the kernel's 12.5 KB of static
+// shared memory stay within the per-CTA limit.
+constexpr int kMaxTopkRow = 786432;
+
+// scores: fp32 [rows][Nc], or bf16 when bf16_scores
+cslc_status launch_topk_rows(const void* scores, bool bf16_scores, int rows_in_buf, int row_begin, int row_end,
                              int B, int L, int Nc, int m, int q_pos0, int topk, int32_t* idx,
                              cudaStream_t stream) {
   if (row_end <= row_begin || B == 0) return CSLC_OK;
+  static int configured_for = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_for != dev) {
+    const int max_dyn = kMaxTopkRow / 4;   // rows above 196,608 entries need more than the default 48 KB
+    cudaFuncSetAttribute(topk_rows_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+    cudaFuncSetAttribute(topk_rows_kernel<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+    configured_for = dev;
+  }
   // mask storage for the launch's longest row (rows see more entries as t grows)
   const int nv_max = n_visible((long long)q_pos0 + row_end - 1, m, Nc);
   const size_t smem = (size_t)((nv_max + TK_SLICE - 1) / TK_SLICE) * (TK_SLICE / 4);
   dim3 grid(row_end - row_begin, B);
-  topk_rows_kernel<<<grid, TOPK_THREADS, smem, stream>>>(scores, rows_in_buf, row_begin, L, Nc, m,
-                                                         q_pos0, topk, idx);
+  if (bf16_scores)
+    topk_rows_kernel<uint16_t><<<grid, TOPK_THREADS, smem, stream>>>(static_cast<const uint16_t*>(scores), rows_in_buf,
+                                                                     row_begin, L, Nc, m, q_pos0, topk, idx);
+  else
+    topk_rows_kernel<float><<<grid, TOPK_THREADS, smem, stream>>>(static_cast<const float*>(scores), rows_in_buf,
+                                                                  row_begin, L, Nc, m, q_pos0, topk, idx);
   return check_launch("topk_rows_kernel");
 }
 

@@ -155,7 +155,8 @@ cslc_status hca_compress_front_end(const cslc_bf16* h, const cslc_bf16* W, const
  *   ws     workspace of csa_indexer_topk_workspace_bytes() bytes (may be NULL
  *          when that is 0).
  * Requires d_I == 64, 1 <= H_I <= 16, 1 <= topk <= 2048, q_pos0 >= 0,
- * Nc <= 45056 (a row of scores is selected in shared memory).
+ * Nc <= 786432 (a row's selection masks, Nc / 4 bytes, stay in shared memory;
+ * the 1M-token CSA context has 262,144 entries).
  */
 size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given);
 cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w,
@@ -169,6 +170,24 @@ cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w,
  * entries of row t are read). */
 cslc_status csa_topk(const float* scores, int B, int L, int Nc, int m, int q_pos0,
                      int topk, int32_t* idx, cslc_stream_t stream);
+
+/* The indexer and top-k with BF16-stored scores (first page §1.4: the
+ * indexer's scores are quantised from FP32 to BF16 to halve the top-k's
+ * traffic). Each score is computed as in csa_indexer_topk (fp32 accumulation)
+ * and rounded to the nearest bf16 (ties to even) before it is stored; idx is
+ * the exact top-k of those bf16 scores under the same rule (ties, which bf16
+ * makes frequent, go to the smaller index). scores [B, L, Nc] bf16 or NULL;
+ * the workspace holds bf16 score blocks (csa_indexer_topk_bf16_workspace_bytes).
+ * Other arguments, requirements and ordering as csa_indexer_topk. */
+size_t csa_indexer_topk_bf16_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given);
+cslc_status csa_indexer_topk_bf16(const cslc_bf16* q_idx, const cslc_bf16* w,
+                                  const cslc_bf16* k_idx, int B, int L, int Nc, int HI,
+                                  int dI, int m, int q_pos0, int topk, cslc_bf16* scores,
+                                  int32_t* idx, void* ws, size_t ws_bytes,
+                                  cslc_stream_t stream);
+/* csa_topk on given bf16 scores [B, L, Nc]. */
+cslc_status csa_topk_bf16(const cslc_bf16* scores, int B, int L, int Nc, int m, int q_pos0,
+                          int topk, int32_t* idx, cslc_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* CSA core attention ("读完这篇…" §三 注意力计算: ordinary attention over the
