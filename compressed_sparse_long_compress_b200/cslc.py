@@ -30,6 +30,7 @@ ABI_SYMBOLS = [
     "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc", "cslc_decode_append",
     "csa_compress_front_end", "hca_compress_front_end",
     "csa_indexer_topk_bf16_workspace_bytes", "csa_indexer_topk_bf16", "csa_topk_bf16",
+    "cslc_testing_set_wait_limits",
 ]
 
 
@@ -79,6 +80,7 @@ def _load():
         "csa_indexer_topk_bf16": (c_int, [P, P, P, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                           P, P, P, c_size_t, P]),
         "csa_topk_bf16": (c_int, [P, c_int, c_int, c_int, c_int, c_int, c_int, P, P]),
+        "cslc_testing_set_wait_limits": (c_int, [ctypes.c_uint64, ctypes.c_uint32]),
         "hca_compress_front_end": (c_int, [P, P, P, c_int, c_int, c_int, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -128,6 +130,15 @@ def abi_version() -> int:
 
 def sync_status(stream=None):
     _check(LIB.cslc_sync_status(_stream(stream)))
+
+
+WAIT_LIMIT_NS_DEFAULT = 2_000_000_000
+WAIT_SLEEP_NS_DEFAULT = 200_000
+
+
+def testing_set_wait_limits(limit_ns: int, sleep_ns: int):
+    """Testing hook: see cslc_testing_set_wait_limits in include/cslc.h."""
+    _check(LIB.cslc_testing_set_wait_limits(int(limit_ns), int(sleep_ns)))
 
 
 # ------------------------------------------------------------- compression

@@ -44,6 +44,10 @@ int sparse_attn_sm100_read_error();
 int dense_attn_sm100_read_error();
 int indexer_sm100_read_error();
 int front_end_sm100_read_error();
+cudaError_t sparse_attn_sm100_set_wait_limits(uint64_t, uint32_t);
+cudaError_t dense_attn_sm100_set_wait_limits(uint64_t, uint32_t);
+cudaError_t indexer_sm100_set_wait_limits(uint64_t, uint32_t);
+cudaError_t front_end_sm100_set_wait_limits(uint64_t, uint32_t);
 cslc_status launch_front_end(const uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int, int, uint16_t*,
                              cudaStream_t);
 size_t decode_topk_workspace_bytes(int, int, int);
@@ -134,6 +138,15 @@ cslc_status cslc_sync_status(cslc_stream_t stream) {
   const int code4 = front_end_sm100_read_error();
   if (code4 != 0)
     return set_error(CSLC_ERR_DEVICE_CHECK, "compressor front end: a pipeline wait timed out (code %d)", code4);
+  return CSLC_OK;
+}
+
+cslc_status cslc_testing_set_wait_limits(uint64_t limit_ns, uint32_t sleep_ns) {
+  cudaError_t e = sparse_attn_sm100_set_wait_limits(limit_ns, sleep_ns);
+  if (e == cudaSuccess) e = dense_attn_sm100_set_wait_limits(limit_ns, sleep_ns);
+  if (e == cudaSuccess) e = indexer_sm100_set_wait_limits(limit_ns, sleep_ns);
+  if (e == cudaSuccess) e = front_end_sm100_set_wait_limits(limit_ns, sleep_ns);
+  if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "cslc_testing_set_wait_limits: %s", cudaGetErrorString(e));
   return CSLC_OK;
 }
 

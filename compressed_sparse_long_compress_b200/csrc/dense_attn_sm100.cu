@@ -112,12 +112,13 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_kv);
       int kv_it = 0;
-      long long tk = 0;
+      long long tk = 0, q_last = -1;   // last tile whose Q load was issued
       bool ok = true;
       for (long long g = blockIdx.x; g < n_qt && ok; g += gridDim.x, ++tk) {
         int b, t0, nkv;
         tile_of(g, b, t0, nkv);
         if (tk >= 1 && !mbar_wait(&bars.q_empty, (uint32_t)((tk - 1) & 1), abortp, errp, ERR_Q_EMPTY)) break;
+        q_last = tk;
         mbar_arrive_expect_tx(&bars.q_full, DA_TILE_BYTES);
         const int qrow = (int)(((long long)b * L + t0) * H);
         tma_load_2d(q_s, &tm_q, 0, qrow, &bars.q_full);
@@ -136,6 +137,13 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
           tma_load_2d(dst + DA_TILE * 128, &tm_kv, 64, krow, &bars.kv_full[stage]);
           ++kv_it;
         }
+      }
+      // loads in flight after an abort land before the CTA leaves (the last
+      // load into each barrier is its latest phase)
+      if (q_last >= 0) mbar_wait_done(&bars.q_full, (uint32_t)(q_last & 1), errp, ERR_Q_FULL);
+      for (int d = 1; d <= DA_STAGES && kv_it - d >= 0; ++d) {
+        const int k2 = kv_it - d;
+        mbar_wait_done(&bars.kv_full[k2 % DA_STAGES], (uint32_t)((k2 / DA_STAGES) & 1), errp, ERR_KV_FULL);
       }
     }
     __syncwarp();
@@ -385,5 +393,7 @@ int dense_attn_sm100_read_error() {
   if (v) cudaMemcpyToSymbol(g_dense_attn_err, &zero, sizeof(int));
   return v;
 }
+
+CSLC_DEFINE_WAIT_LIMIT_SETTER(dense_attn_sm100_set_wait_limits)
 
 }  // namespace cslc

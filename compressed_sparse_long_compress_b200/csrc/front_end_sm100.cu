@@ -341,4 +341,6 @@ int front_end_sm100_read_error() {
   return v;
 }
 
+CSLC_DEFINE_WAIT_LIMIT_SETTER(front_end_sm100_set_wait_limits)
+
 }  // namespace cslc

@@ -354,4 +354,6 @@ int indexer_sm100_read_error() {
   return v;
 }
 
+CSLC_DEFINE_WAIT_LIMIT_SETTER(indexer_sm100_set_wait_limits)
+
 }  // namespace cslc

@@ -51,20 +51,27 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far beyond any legitimate wait
-constexpr uint32_t kSleepHintNs = 200000;          // a waiting thread re-checks the abort flag every <= 0.2 ms
+constexpr uint64_t kWaitLimitNs = CSLC_WAIT_LIMIT_NS_DEFAULT;   // 2 s: far beyond any legitimate wait
+constexpr uint32_t kSleepHintNs = CSLC_WAIT_SLEEP_NS_DEFAULT;    // a waiting thread re-checks the abort flag every <= 0.2 ms
+
+// The limits a pipeline wait uses (one copy per translation unit; tests
+// lower them through cslc_testing_set_wait_limits to make waits run out).
+static __device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+static __device__ uint32_t g_sleep_hint_ns = kSleepHintNs;
 
 // Waits for the phase of `bar` with the given parity to complete. Gives up
-// after kWaitLimitNs or as soon as another role raised *abort; on giving up
-// it raises *abort, records `code` in *err (first error wins) and returns false.
+// after g_wait_limit_ns or as soon as another role raised *abort; on giving
+// up it raises *abort, records `code` in *err (first error wins) and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
                                           int code) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_ns();
+  const uint64_t limit = g_wait_limit_ns;
+  const uint32_t hint = g_sleep_hint_ns;
   while (true) {
-    if (mbar_test_sleep(bar, parity, kSleepHintNs)) return true;
+    if (mbar_test_sleep(bar, parity, hint)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit) {
       *abort = 1;
       atomicCAS(err, 0, code);
       return false;
@@ -72,9 +79,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Waits (time-bounded, ignoring the abort flag) for work that completes on
-// its own -- tensor-core products or TMA copies already issued -- before the
-// CTA releases what they use. Records `code` in *err on a timeout.
+// Waits (time-bounded by the fixed kWaitLimitNs, ignoring the abort flag) for
+// work that completes on its own -- tensor-core products or TMA copies already
+// issued -- before the CTA releases what they use. Records `code` in *err on
+// a timeout.
 __device__ __forceinline__ bool mbar_wait_done(uint64_t* bar, uint32_t parity, int* err, int code) {
   const uint64_t t0 = global_ns();
   while (!mbar_test_sleep(bar, parity, kSleepHintNs)) {
@@ -253,6 +261,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte swizzled block.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// Host: sets this translation unit's wait limits (see cslc_testing_set_wait_limits).
+#define CSLC_DEFINE_WAIT_LIMIT_SETTER(fn)                                            \
+  cudaError_t fn(uint64_t limit_ns, uint32_t sleep_ns) {                            \
+    cudaError_t e = cudaMemcpyToSymbol(sm100::g_wait_limit_ns, &limit_ns, sizeof(limit_ns)); \
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(sm100::g_sleep_hint_ns, &sleep_ns, sizeof(sleep_ns)); \
+    return e;                                                                        \
+  }
 
 // Host: 2-D bf16 tensor map (rows x cols, row pitch in bytes) with a box of
 // box_rows x box_cols elements and 128-byte swizzle; false on failure.

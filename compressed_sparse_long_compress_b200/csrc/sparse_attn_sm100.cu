@@ -606,4 +606,6 @@ int sparse_attn_sm100_read_error() {
   return v;
 }
 
+CSLC_DEFINE_WAIT_LIMIT_SETTER(sparse_attn_sm100_set_wait_limits)
+
 }  // namespace cslc

@@ -52,6 +52,8 @@ extern "C" {
 #endif
 
 #define CSLC_ABI_VERSION 1
+#define CSLC_WAIT_LIMIT_NS_DEFAULT 2000000000ull   /* a pipeline wait gives up after 2 s */
+#define CSLC_WAIT_SLEEP_NS_DEFAULT 200000u         /* a waiting thread re-checks every <= 0.2 ms */
 
 typedef uint16_t cslc_bf16;              /* raw bfloat16 bits */
 typedef struct CUstream_st* cslc_stream_t; /* the same handle as cudaStream_t */
@@ -76,6 +78,17 @@ const char* cslc_last_error(void);
 /* Waits for `stream`, then reports (and clears) any error a kernel recorded in
  * its device-side status word; returns CSLC_OK when none. */
 cslc_status cslc_sync_status(cslc_stream_t stream);
+
+/* Testing hook (no counterpart on the pages): the time after which a
+ * pipelined kernel's wait gives up, and how long a waiting thread sleeps
+ * between checks, for the kernels launched after the call on the current
+ * device (defaults CSLC_WAIT_LIMIT_NS_DEFAULT, CSLC_WAIT_SLEEP_NS_DEFAULT).
+ * A wait that gives up raises its CTA's abort: every role of the CTA leaves
+ * its loop, products and copies already issued complete, TMEM is released,
+ * and cslc_sync_status reports CSLC_ERR_DEVICE_CHECK; later calls run
+ * normally. Synchronises with the legacy default stream. Tests use it to make
+ * waits run out on small grids; production code leaves the defaults. */
+cslc_status cslc_testing_set_wait_limits(uint64_t limit_ns, uint32_t sleep_ns);
 
 /* ------------------------------------------------------------------------ */
 /* Compression ("读完这篇你就搞懂 DeepSeek v4 了", §三 压缩机制; first page §1.1 工程细节)
