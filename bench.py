@@ -633,6 +633,23 @@ def profile_case(name):
         x = W.front_end_inputs(s, 6, device=dev)
         for _ in range(2):
             C.compress_front_end(x["h"], x["W"], x["pos_bias"], s.m, True)
+    elif name == "dense_attn_steady":   # the last 16384 query rows of the 1,048,576-token HCA layer
+        L, H, n_c = 16384, 64, 8192
+        q = W.randn_bf16((1, L, H, 128), 1, device=dev)
+        e = W.randn_bf16((1, n_c, 128), 2, device=dev, std=0.4)
+        out = torch.empty_like(q)
+        for _ in range(2):
+            C.hca_dense_attn(q, e, m_prime=128, scale=1 / math.sqrt(128), q_pos0=128 * n_c - L, out=out)
+    elif name in ("compress_L65536", "compress_hca_L1M"):   # the two prefill workloads' compression
+        L, m, overlap = (65536, 4, True) if name == "compress_L65536" else (1 << 20, 128, False)
+        c = W.randn_bf16((1, L, 128), 8, device=dev)
+        z = W.randn_bf16((1, L, 128), 9, device=dev)
+        bias = W.randn_bf16((2 * m if overlap else m, 128), 10, device=dev, std=0.1)
+        for _ in range(2):
+            if overlap:
+                C.csa_compress(c, z, bias, m=m)
+            else:
+                C.hca_compress(c, z, bias, m_prime=m)
     elif name in ("csa_decode", "hybrid_decode"):   # the full decode workloads (about 1-1.4 GB on the device)
         wl = Decode(C, dev, 0, name)
         for _ in range(2):
@@ -843,7 +860,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of timed oracle work for the headline's CPU baseline (a third for each secondary)")
     ap.add_argument("--profile-case", default=None, choices=["sparse_attn_L8192", "dense_attn_L65536", "topk_L8192", "indexer_L8192",
-                                                              "csa_decode", "hybrid_decode", "front_end_L16384"],
+                                                              "csa_decode", "hybrid_decode", "front_end_L16384", "dense_attn_steady",
+                                                              "compress_L65536", "compress_hca_L1M"],
                     help="run one small kernel case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:
@@ -870,7 +888,6 @@ def main():
             r = measure(name, C, args, world, rank, local, peaks, flush, with_e2e=False, min_timed_ms=500.0)
             secondary[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "kernel_ms", "roofline",
                                                   "clocks", "config", "steps")}
-            head["gpu_launches"] += r["gpu_launches"] * 0   # reported per workload below
             secondary[name]["gpu_launches"] = r["gpu_launches"]
         secondary["indexer_topk_bf16_scores"] = measure_indexer_bf16(C, torch.device("cuda", local), flush)
 
@@ -878,7 +895,8 @@ def main():
     if rank == 0 and world == 1:
         cpu = cpu_baseline_entry(args.workload, budget_s=args.cpu_budget, one_thread_s=args.cpu_budget / 4)
         for name in secondary:
-            secondary[name]["cpu_baseline"] = cpu_baseline_entry(name, budget_s=args.cpu_budget / 3)
+            if name in W.WORKLOADS:   # the bf16-score entry is a variant of the headline's indexer
+                secondary[name]["cpu_baseline"] = cpu_baseline_entry(name, budget_s=args.cpu_budget / 3)
 
     if rank == 0:
         line = {"metric": "CSA+HCA prefill tokens/s and 1M-ctx decode us/step; % of TC/HBM roofline",
