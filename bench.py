@@ -666,11 +666,11 @@ def profile_case(name):
 # kernel source is the one that was measured.
 MEASURED_TRAFFIC = {
     "sparse": {"src": "sparse_attn_sm100.cu",
-               "sha256": "ed29a584fc1f57bf61ff5e3eafef79629f9b0007f8da200babf5e202cc1151b0",
-               "bytes_per_token": (172.033792e6 + 102.792960e6) / 8192},
+               "sha256": "aef8a553ca588a590c3111df77e6cb1aedbe1e808e09b36955548148c2ee4bc2",
+               "bytes_per_token": (172.444416e6 + 101.987328e6) / 8192},
     "dense": {"src": "dense_attn_sm100.cu",
-              "sha256": "73e711b1c99da856d8e4ebac26f96470f4f5e0eca29bcf506e33aa08a9f8f1f0",
-              "bytes_per_token": (1.074094e9 + 1.024188e9) / 65536},
+              "sha256": "288507378b3c15bc7d245eaa6a83a4535775efaf20ba08db79a0d8c7654f0086",
+              "bytes_per_token": (271.271424e6 + 221.559552e6) / 16384},
 }
 
 
