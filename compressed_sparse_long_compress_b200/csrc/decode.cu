@@ -28,6 +28,9 @@
 //                          / PV run for all heads
 //   decode_combine_kernel  merges the splits with their max / sum statistics
 //                          (two thread groups, each over half of the splits)
+//   decode_tail_kernel     for large batches, select + finalize + attention +
+//                          combine of a CSA layer in one launch of one
+//                          thread-block cluster per sequence (see its comment)
 // The layers of a step are independent: layer 0 runs on the caller's stream,
 // the others on internal streams forked from it and joined back with events,
 // each with its own workspace slice. Inside a layer the kernels after the
@@ -764,6 +767,625 @@ __global__ void __launch_bounds__(2 * kD) decode_combine_kernel(const float* __r
   }
 }
 
+// ------------------------------------------------- fused layer tail (clusters)
+//
+// One thread-block cluster of CL CTAs per sequence runs everything after the
+// index scan of a CSA layer (and the whole of an HCA layer) in one launch,
+// exchanging through distributed shared memory instead of global round trips:
+//   selection  every CTA finds the threshold bin from the scan's histogram
+//              and classifies its 1/CL of the scores: above the bin =
+//              selected (kept in its shared memory), inside = candidate
+//              (kept in its own slice of the candidate buffer);
+//   choice     exact radix select among all candidates by 8-bit digits of
+//              (score key, reversed index): each CTA histograms its own
+//              candidates and sums all CTAs' histograms, so every CTA takes
+//              the same digit with no further exchange;
+//   order      each CTA marks its selected entries in a bitmap of its range;
+//              a cluster scan of the counts places them, ascending, in the
+//              index list held in CTA 0's shared memory (and idx_out);
+//   attention  CTA r takes slots [r*S, (r+1)*S) of the list, as
+//              decode_attn_kernel does per chunk; with H <= 64 two warp groups
+//              take alternate 64-entry tiles and merge before publishing;
+//   combine    every CTA's partial (max, sum, O) stays in its shared memory;
+//              CTA r merges heads [r*H/CL, (r+1)*H/CL) over the cluster.
+// Every CTA passes the same cluster barriers in the same order: each branch
+// around one depends on per-sequence values or on sums every CTA computes
+// identically. The CTAs of a cluster are co-scheduled by the hardware.
+
+constexpr int TAIL_THREADS = 256;
+constexpr int TAIL_BM_WORDS = 4096;   // bitmap words per CTA: ranges up to 131,072 entries
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire;\n" ::: "memory");
+}
+// the address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void dsmem_st_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Dynamic shared memory of the tail kernel: the index list (CTA 0's is the
+// cluster's), then one region used in turn by the selection, the attention
+// and the combine.
+__host__ __device__ constexpr size_t tail_sel_bytes() { return 2 * 256 * 4 + MAX_TOPK * 4 + TAIL_BM_WORDS * 4; }
+constexpr int TAIL_NBUF = 4;          // chunks of stored entries in flight per CTA
+__host__ __device__ constexpr size_t tail_attn_bytes(int H) {
+  return (size_t)H * 256 + SPLIT * 256 + TAIL_NBUF * (size_t)SPLIT * (kNope + kRope * 2 + 4);
+}
+__host__ __device__ constexpr size_t tail_smem_bytes(int H) {
+  return MAX_TOPK * 4 + (tail_sel_bytes() > tail_attn_bytes(H) ? tail_sel_bytes() : tail_attn_bytes(H));
+}
+
+template <bool SPARSE, int CL>
+__global__ void __launch_bounds__(TAIL_THREADS) decode_tail_kernel(
+    const uint16_t* __restrict__ q, const uint8_t* __restrict__ nope, const uint16_t* __restrict__ rope,
+    const float* __restrict__ kv_scale, const int32_t* __restrict__ n_entries, int n_max,
+    const float* __restrict__ scores, const uint32_t* __restrict__ ghist, uint2* __restrict__ cand, int topk,
+    int H, float scale_log2, int32_t* __restrict__ idx_out, uint16_t* __restrict__ out) {
+  constexpr int ST_BYTES = SPLIT * (kNope + kRope * 2 + 4);
+  extern __shared__ __align__(128) uint8_t smem[];
+  int32_t* list = reinterpret_cast<int32_t*>(smem);   // [MAX_TOPK], read from CTA 0 by all
+  uint8_t* work = smem + MAX_TOPK * 4;
+  __shared__ uint32_t pub[4];                          // read by the other CTAs
+  __shared__ int s_thr[2], s_nab, s_ncand, s_base, s_tot[2], bc[3];
+  __shared__ uint32_t htot[256];
+  __shared__ uint32_t wtot[TAIL_THREADS / 32];
+  __shared__ int32_t ent_buf[2 * TAIL_NBUF][SPLIT];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const int b = blockIdx.y;
+  pdl_wait();
+  const int n = max(0, min(n_entries[b], n_max));
+  const bool select = SPARSE && n > topk;
+  const int k_eff = SPARSE ? min(topk, n) : n;
+
+  if (SPARSE && !select && idx_out != nullptr)
+    for (int j = (int)rank * TAIL_THREADS + tid; j < topk; j += CL * TAIL_THREADS)
+      idx_out[(size_t)b * topk + j] = j < n ? j : -1;
+
+  if (select) {
+    const int R = ((n + CL - 1) / CL + 31) & ~31;     // entries per CTA (multiple of 32)
+    const int e_lo = (int)rank * R, e_hi = min(n, e_lo + R);
+    uint32_t* hist2 = reinterpret_cast<uint32_t*>(work);                            // [2][256]
+    int32_t* above_l = reinterpret_cast<int32_t*>(work + 2 * 256 * 4);                // [MAX_TOPK]
+    uint32_t* bm = reinterpret_cast<uint32_t*>(work + 2 * 256 * 4 + MAX_TOPK * 4);    // [R / 32]
+    if (tid == 0) { s_nab = 0; s_ncand = 0; s_thr[0] = HIST_BINS; s_thr[1] = 0; }
+    find_threshold_bin(ghist + (size_t)b * HIST_BINS, topk, &s_thr[0], &s_thr[1]);
+    const uint32_t T = (uint32_t)s_thr[0];
+    uint2* my_cand = cand + (size_t)b * n_max + e_lo;
+    const float* srow = scores + (size_t)b * n_max;
+    const unsigned lt = (1u << lane) - 1u;
+    // rounds of 32 scores per thread: flag masks (above the bin / in it),
+    // one block scan of the counts, then each thread writes its scores' entry
+    // numbers (above: this CTA's list; in the bin: its candidate slice)
+    const bool vec = (n_max & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
+    // element k of this thread in the round at `base` (16-byte loads: 4 consecutive per load)
+    auto e_of = [&](int base, int k) {
+      return vec ? base + 4 * ((k >> 2) * TAIL_THREADS + tid) + (k & 3) : base + k * TAIL_THREADS + tid;
+    };
+    int run_above = 0, run_cand = 0;   // this CTA's counts so far (the same in every thread)
+    for (int base = e_lo; base < e_hi; base += TAIL_THREADS * 32) {
+      float val[32];
+      if (vec) {
+        const float4* s4 = reinterpret_cast<const float4*>(srow);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = e_of(base, 4 * i);
+          // rows are 16-byte aligned and e is a multiple of 4, so a load that
+          // starts before e_hi stays inside the row (n_max is a multiple of 4)
+          const float4 v = e < e_hi ? s4[e >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+          val[4 * i] = v.x; val[4 * i + 1] = v.y; val[4 * i + 2] = v.z; val[4 * i + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int e = e_of(base, k);
+          val[k] = e < e_hi ? srow[e] : 0.f;
+        }
+      }
+      uint32_t fa = 0u, fc = 0u;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const uint32_t bin = float_key(val[k]) >> HIST_SHIFT;
+        const bool in = e_of(base, k) < e_hi;
+        if (in && bin > T) fa |= 1u << k;
+        if (in && bin == T) fc |= 1u << k;
+      }
+      const uint32_t mine = ((uint32_t)__popc(fa) << 16) | (uint32_t)__popc(fc);
+      uint32_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane == 31) wtot[warp] = incl;
+      __syncthreads();
+      uint32_t before = 0u, total = 0u;
+#pragma unroll
+      for (int w = 0; w < TAIL_THREADS / 32; ++w) {
+        const uint32_t t = wtot[w];
+        if (w < warp) before += t;
+        total += t;
+      }
+      const uint32_t excl = before + incl - mine;
+      int pa = run_above + (int)(excl >> 16), pc = run_cand + (int)(excl & 0xffffu);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        if ((fa >> k) & 1u) {
+          if (pa < MAX_TOPK) above_l[pa] = e_of(base, k);
+          ++pa;
+        }
+        if ((fc >> k) & 1u) my_cand[pc++] = make_uint2(float_key(val[k]), (uint32_t)e_of(base, k));
+      }
+      run_above += (int)(total >> 16);
+      run_cand += (int)(total & 0xffffu);
+      __syncthreads();   // wtot is rewritten by the next round
+    }
+    if (tid == 0) { s_nab = run_above; s_ncand = run_cand; }
+    __syncthreads();
+    if (tid == 0) { pub[0] = (uint32_t)s_nab; pub[1] = (uint32_t)s_ncand; }
+    cluster_sync_all();   // counts published
+    if (warp == 0) {
+      uint32_t a = 0u, c = 0u;
+      if (lane < CL) {
+        a = dsmem_ld_u32(dsmem_addr(&pub[0], lane));
+        c = dsmem_ld_u32(dsmem_addr(&pub[1], lane));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+      }
+      if (lane == 0) { s_tot[0] = (int)a; s_tot[1] = (int)c; }
+    }
+    __syncthreads();
+    const int nc = s_ncand;
+
+    // exact choice among the candidates: they share the bin's key bits, so the
+    // digits start below them (8-bit digits, a last 4-bit one)
+    constexpr int FIXED = 64 - (32 - HIST_SHIFT);
+    uint64_t prefix = (uint64_t)T << FIXED, mask = ~0ull << FIXED;
+    int remaining = topk - s_tot[0];
+    bool take_all = (s_tot[1] == remaining);
+    int pass = 0;
+    for (int shift = FIXED - 8; shift > -8 && !take_all; shift -= 8, ++pass) {
+      const int sh = shift < 0 ? 0 : shift;
+      const uint32_t dmask = shift < 0 ? (0xffu >> -shift) : 0xffu;
+      uint32_t* h = hist2 + (pass & 1) * 256;
+      h[tid] = 0u;   // TAIL_THREADS == 256 digits
+      __syncthreads();
+      for (int i = tid; i < nc; i += TAIL_THREADS) {
+        const uint64_t k = cand_key(my_cand[i]);
+        if ((k & mask) == prefix) atomicAdd(&h[(uint32_t)(k >> sh) & dmask], 1u);
+      }
+      __syncthreads();
+      cluster_sync_all();   // every CTA's histogram of this digit is complete
+      uint32_t sum = 0u;
+      for (int r = 0; r < CL; ++r) sum += dsmem_ld_u32(dsmem_addr(&h[tid], r));
+      htot[tid] = sum;
+      __syncthreads();
+      if (warp == 0) {
+        // a default every CTA shares, so that the pass count stays the same
+        // across the cluster even if no digit were found
+        if (lane == 0) { bc[0] = 0; bc[1] = 0; bc[2] = -1; }
+        __syncwarp();
+        uint32_t cnt[8], ls = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { cnt[j] = htot[255 - 8 * lane - j]; ls += cnt[j]; }
+        uint32_t incl = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const uint32_t excl = incl - ls;
+        if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
+          uint32_t above = excl;
+          for (int j = 0; j < 8; ++j) {
+            if (above + cnt[j] >= (uint32_t)remaining) {
+              bc[0] = 255 - 8 * lane - j; bc[1] = (int)above; bc[2] = (int)cnt[j];
+              break;
+            }
+            above += cnt[j];
+          }
+        }
+      }
+      __syncthreads();
+      remaining -= bc[1];
+      prefix |= (uint64_t)bc[0] << sh;
+      mask |= (uint64_t)dmask << sh;
+      if (bc[2] == remaining) take_all = true;
+      __syncthreads();   // bc and htot are rewritten by the next pass
+    }
+
+    // this CTA's selected entries, in ascending order, into CTA 0's list
+    const int words = R >> 5;
+    for (int x = tid; x < words; x += TAIL_THREADS) bm[x] = 0u;
+    __syncthreads();
+    const int nab = min(s_nab, MAX_TOPK);
+    for (int j = tid; j < nab; j += TAIL_THREADS) {
+      const int e = above_l[j] - e_lo;
+      atomicOr(&bm[e >> 5], 1u << (e & 31));
+    }
+    for (int i = tid; i < nc; i += TAIL_THREADS) {
+      const uint2 c = my_cand[i];
+      if ((cand_key(c) & mask) >= prefix) {
+        const int e = (int)c.y - e_lo;
+        atomicOr(&bm[e >> 5], 1u << (e & 31));
+      }
+    }
+    __syncthreads();
+    const int wpt = (words + TAIL_THREADS - 1) / TAIL_THREADS;   // words per thread
+    int cnt = 0;
+    for (int k = 0; k < wpt; ++k) {
+      const int x = tid * wpt + k;
+      if (x < words) cnt += __popc(bm[x]);
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wtot[warp] = (uint32_t)incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < TAIL_THREADS / 32; ++w) {
+      const int t = (int)wtot[w];
+      if (w < warp) before += t;
+      total += t;
+    }
+    if (tid == 0) pub[2] = (uint32_t)total;
+    cluster_sync_all();   // selected counts published
+    if (warp == 0) {
+      int c = (lane < (int)rank) ? (int)dsmem_ld_u32(dsmem_addr(&pub[2], lane)) : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+      if (lane == 0) s_base = c;
+    }
+    __syncthreads();
+    int pos = s_base + before + incl - cnt;
+    const uint32_t list0 = dsmem_addr(list, 0);
+    for (int k = 0; k < wpt; ++k) {
+      const int x = tid * wpt + k;
+      uint32_t wv = x < words ? bm[x] : 0u;
+      while (wv) {
+        const int e = e_lo + x * 32 + (__ffs(wv) - 1);
+        if (pos < topk) {
+          dsmem_st_u32(list0 + 4u * (uint32_t)pos, (uint32_t)e);
+          if (idx_out != nullptr) idx_out[(size_t)b * topk + pos] = e;
+        }
+        ++pos;
+        wv &= wv - 1u;
+      }
+    }
+  }
+  cluster_sync_all();   // the list is complete; the selection's scratch is free
+
+  // ---- attention over this CTA's slots
+  uint8_t* q_s = work;                 // [H][256 B]
+  uint8_t* kv_s = work + H * 256;      // [SPLIT][256 B] dequantised entries
+  uint8_t* st_base = kv_s + SPLIT * 256;
+  const int S = ((k_eff + CL - 1) / CL + DTILE - 1) / DTILE * DTILE;
+  const int slot0 = (int)rank * S;
+  const int slot_end = min(k_eff, slot0 + S);
+  const int n_chunks = slot_end > slot0 ? (slot_end - slot0 + SPLIT - 1) / SPLIT : 0;
+  const uint32_t list0 = dsmem_addr(list, 0);
+  const int wpg = H / 16;              // warps per group; a warp owns 16 heads
+  const int G = H <= 64 ? 2 : 1;       // groups taking alternate tiles
+  const int grp = warp / wpg, lw = warp - grp * wpg;
+  const bool mma_warp = grp < G;
+  const int g = lane >> 2, tq = lane & 3;
+
+  // chunk c's entry indices go to ent_buf[c % (2 NBUF)] and its stored
+  // entries to staging buffer c % NBUF; NBUF chunks are in flight at once
+  auto fill_ent = [&](int c) {
+    for (int j = tid; j < SPLIT; j += TAIL_THREADS) {
+      const int slot = slot0 + c * SPLIT + j;
+      int e = -1;
+      if (slot < slot_end) e = select ? (int)dsmem_ld_u32(list0 + 4u * (uint32_t)slot) : slot;
+      if (e >= n) e = -1;
+      ent_buf[c % (2 * TAIL_NBUF)][j] = e;
+    }
+  };
+  constexpr int PIECES = kNope / 16 + (kRope * 2) / 16 + 1;
+  auto stage_chunk = [&](int c) {
+    uint8_t* st_nope = st_base + (c % TAIL_NBUF) * ST_BYTES;
+    uint8_t* st_rope = st_nope + SPLIT * kNope;
+    float* st_scale = reinterpret_cast<float*>(st_rope + SPLIT * kRope * 2);
+    const int32_t* ent = ent_buf[c % (2 * TAIL_NBUF)];
+    for (int x = tid; x < SPLIT * PIECES; x += TAIL_THREADS) {
+      const int row = x / PIECES, pc = x - row * PIECES;
+      const int e = ent[row];
+      const size_t er = (size_t)b * n_max + (e < 0 ? 0 : e);
+      if (pc < kNope / 16)
+        cp_async16(smem_u32(st_nope + row * kNope + pc * 16), nope + er * kNope + pc * 16, e >= 0);
+      else if (pc < PIECES - 1)
+        cp_async16(smem_u32(st_rope + row * (kRope * 2) + (pc - kNope / 16) * 16),
+                   reinterpret_cast<const uint8_t*>(rope + er * kRope) + (pc - kNope / 16) * 16, e >= 0);
+      else
+        cp_async4(smem_u32(st_scale + row), kv_scale + er, e >= 0);
+    }
+    cp_async_commit();
+  };
+  const int n_pre = min(n_chunks, TAIL_NBUF);
+  for (int c = 0; c < n_pre; ++c) fill_ent(c);
+  __syncthreads();
+  for (int c = 0; c < n_pre; ++c) {
+    if (c == 0)   // the queries travel in the first chunk's group of copies
+      for (int x = tid; x < H * 16; x += TAIL_THREADS) {
+        const int chunk = x & 15, row = x >> 4;
+        cp_async16(smem_u32(q_s + swz(row, chunk, 256)), q + ((size_t)b * H + row) * kD + chunk * 8, true);
+      }
+    stage_chunk(c);
+  }
+  uint32_t qf[8][4];
+  float o[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+
+  for (int c = 0; c < n_chunks; ++c) {
+    // groups committed so far: chunks 0 .. min(n_chunks, c + NBUF) - 1; chunk c's must be complete
+    const int pending = min(n_chunks, c + TAIL_NBUF) - c - 1;
+    if (pending >= 3) cp_async_wait<3>();
+    else if (pending == 2) cp_async_wait<2>();
+    else if (pending == 1) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    if (c + TAIL_NBUF < n_chunks) fill_ent(c + TAIL_NBUF);   // its ent slot was last used by chunk c - NBUF
+    __syncthreads();
+    if (c == 0 && mma_warp) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int row = lw * 16 + (lane & 15);
+        const int chunk = ks * 2 + (lane >> 4);
+        ldsm_x4(smem_u32(q_s + swz(row, chunk, 256)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+      }
+    }
+    const int32_t* ent = ent_buf[c % (2 * TAIL_NBUF)];
+    const int s0 = slot0 + c * SPLIT;
+    {
+      const uint8_t* st_nope = st_base + (c % TAIL_NBUF) * ST_BYTES;
+      const uint8_t* st_rope = st_nope + SPLIT * kNope;
+      const float* st_scale = reinterpret_cast<const float*>(st_rope + SPLIT * kRope * 2);
+      for (int x = tid; x < SPLIT * 16; x += TAIL_THREADS) {
+        const int chunk = x & 15, row = x >> 4;
+        uint4 v;
+        if (chunk < 8) {
+          const uint2 c8 = *reinterpret_cast<const uint2*>(st_nope + row * kNope + chunk * 8);
+          const float sc = st_scale[row];
+          const uint32_t cw[2] = {c8.x, c8.y};
+          uint32_t ow[4];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] & 0xffffu), __NV_E4M3);
+            const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[k] >> 16), __NV_E4M3);
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+            ow[2 * k] = pack_bf16x2(f01.x * sc, f01.y * sc);
+            ow[2 * k + 1] = pack_bf16x2(f23.x * sc, f23.y * sc);
+          }
+          v = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        } else {
+          v = *reinterpret_cast<const uint4*>(st_rope + row * (kRope * 2) + (chunk - 8) * 16);
+        }
+        *reinterpret_cast<uint4*>(kv_s + swz(row, chunk, 256)) = v;
+      }
+    }
+    __syncthreads();
+    if (c + TAIL_NBUF < n_chunks) stage_chunk(c + TAIL_NBUF);   // into the buffer just dequantised
+    if (mma_warp) {
+      for (int tile = grp; tile < SPLIT / DTILE; tile += G) {
+        const int t0 = tile * DTILE;
+        if (s0 + t0 >= slot_end) break;
+        const uint8_t* kv_t = kv_s + t0 * 256;
+        float sc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sc[i][j] = 0.f;
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            uint32_t b0, b1, b2, b3;
+            const int row = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+            const int chunk = ks * 2 + ((lane >> 3) & 1);
+            ldsm_x4(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
+            mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
+            mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+          }
+        }
+        float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const bool valid = ent[t0 + nt * 8 + 2 * tq + j] >= 0;
+            const float v0 = valid ? sc[nt][j] * scale_log2 : -INFINITY;
+            const float v1 = valid ? sc[nt][2 + j] * scale_log2 : -INFINITY;
+            sc[nt][j] = v0;
+            sc[nt][2 + j] = v1;
+            tmax[0] = fmaxf(tmax[0], v0);
+            tmax[1] = fmaxf(tmax[1], v1);
+          }
+        }
+        float alpha[2], mnew[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
+          tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
+          mnew[r] = fmaxf(mrow[r], tmax[r]);
+          alpha[r] = mrow[r] == -INFINITY ? 0.f : dec_ex2(mrow[r] - mnew[r]);
+          mrow[r] = mnew[r];
+        }
+        float psum[2] = {0.f, 0.f};
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = j >> 1;
+            const float p = mnew[r] == -INFINITY ? 0.f : dec_ex2(sc[nt][j] - mnew[r]);
+            sc[nt][j] = p;
+            psum[r] += p;
+          }
+        }
+        lrow[0] = lrow[0] * alpha[0] + psum[0];
+        lrow[1] = lrow[1] * alpha[1] + psum[1];
+#pragma unroll
+        for (int dn = 0; dn < 16; ++dn) {
+          o[dn][0] *= alpha[0]; o[dn][1] *= alpha[0];
+          o[dn][2] *= alpha[1]; o[dn][3] *= alpha[1];
+        }
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          uint32_t pa[4];
+          pa[0] = pack_bf16x2(sc[2 * ks][0], sc[2 * ks][1]);
+          pa[1] = pack_bf16x2(sc[2 * ks][2], sc[2 * ks][3]);
+          pa[2] = pack_bf16x2(sc[2 * ks + 1][0], sc[2 * ks + 1][1]);
+          pa[3] = pack_bf16x2(sc[2 * ks + 1][2], sc[2 * ks + 1][3]);
+#pragma unroll
+          for (int dp = 0; dp < 8; ++dp) {
+            uint32_t b0, b1, b2, b3;
+            const int row = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+            const int chunk = dp * 2 + (lane >> 4);
+            ldsm_x4_t(smem_u32(kv_t + swz(row, chunk, 256)), b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * dp], pa, b0, b1);
+            mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+          }
+        }
+      }
+    }
+    __syncthreads();   // kv_s and ent_buf are rewritten for the next chunk
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
+    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
+  }
+
+  // ---- this CTA's partial: group 1 hands its rows to group 0, which merges
+  float* po_s = reinterpret_cast<float*>(work);   // [H][kD]
+  float* ml_s = po_s + (size_t)H * kD;            // [H][2]
+  const int h0 = lw * 16 + g, h1 = h0 + 8;
+  __syncthreads();   // the attention's shared memory is free
+  if (mma_warp && grp == 1) {
+#pragma unroll
+    for (int dn = 0; dn < 16; ++dn) {
+      const int col = dn * 8 + 2 * tq;
+      *reinterpret_cast<float2*>(po_s + (size_t)h0 * kD + col) = make_float2(o[dn][0], o[dn][1]);
+      *reinterpret_cast<float2*>(po_s + (size_t)h1 * kD + col) = make_float2(o[dn][2], o[dn][3]);
+    }
+    if (tq == 0) {
+      ml_s[2 * h0] = mrow[0]; ml_s[2 * h0 + 1] = lrow[0];
+      ml_s[2 * h1] = mrow[1]; ml_s[2 * h1 + 1] = lrow[1];
+    }
+  }
+  __syncthreads();
+  if (mma_warp && grp == 0) {
+    if (G == 2) {
+      const float m1[2] = {ml_s[2 * h0], ml_s[2 * h1]}, l1[2] = {ml_s[2 * h0 + 1], ml_s[2 * h1 + 1]};
+      float a0[2], a1[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float M = fmaxf(mrow[r], m1[r]);
+        a0[r] = mrow[r] == -INFINITY ? 0.f : exp2f(mrow[r] - M);
+        a1[r] = m1[r] == -INFINITY ? 0.f : exp2f(m1[r] - M);
+        lrow[r] = lrow[r] * a0[r] + l1[r] * a1[r];
+        mrow[r] = M;
+      }
+#pragma unroll
+      for (int dn = 0; dn < 16; ++dn) {
+        const int col = dn * 8 + 2 * tq;
+        const float2 p0 = *reinterpret_cast<const float2*>(po_s + (size_t)h0 * kD + col);
+        const float2 p1 = *reinterpret_cast<const float2*>(po_s + (size_t)h1 * kD + col);
+        o[dn][0] = o[dn][0] * a0[0] + p0.x * a1[0];
+        o[dn][1] = o[dn][1] * a0[0] + p0.y * a1[0];
+        o[dn][2] = o[dn][2] * a0[1] + p1.x * a1[1];
+        o[dn][3] = o[dn][3] * a0[1] + p1.y * a1[1];
+      }
+      __syncwarp();   // every lane has read its twin's (max, sum) before lane tq == 0 rewrites them
+    }
+#pragma unroll
+    for (int dn = 0; dn < 16; ++dn) {
+      const int col = dn * 8 + 2 * tq;
+      *reinterpret_cast<float2*>(po_s + (size_t)h0 * kD + col) = make_float2(o[dn][0], o[dn][1]);
+      *reinterpret_cast<float2*>(po_s + (size_t)h1 * kD + col) = make_float2(o[dn][2], o[dn][3]);
+    }
+    if (tq == 0) {
+      ml_s[2 * h0] = mrow[0]; ml_s[2 * h0 + 1] = lrow[0];
+      ml_s[2 * h1] = mrow[1]; ml_s[2 * h1 + 1] = lrow[1];
+    }
+  }
+  cluster_sync_all();   // every CTA's partial is in its shared memory
+
+  // ---- combine: CTA r writes heads [r*H/CL, (r+1)*H/CL), four dims per item
+  const int hpc = H / CL;
+  for (int x = tid; x < hpc * (kD / 4); x += TAIL_THREADS) {
+    const int h = (int)rank * hpc + x / (kD / 4), d4 = (x % (kD / 4)) * 4;
+    float ms[CL], ls[CL];
+    float4 os[CL];
+#pragma unroll
+    for (int r = 0; r < CL; ++r) {
+      ms[r] = dsmem_ld_f32(dsmem_addr(ml_s + 2 * h, r));
+      ls[r] = dsmem_ld_f32(dsmem_addr(ml_s + 2 * h + 1, r));
+      os[r] = dsmem_ld_f32x4(dsmem_addr(po_s + (size_t)h * kD + d4, r));
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, ms[r]);
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int r = 0; r < CL; ++r) {
+        if (ms[r] == -INFINITY) continue;
+        const float f = exp2f(ms[r] - M);
+        den = fmaf(f, ls[r], den);
+        num.x = fmaf(f, os[r].x, num.x);
+        num.y = fmaf(f, os[r].y, num.y);
+        num.z = fmaf(f, os[r].z, num.z);
+        num.w = fmaf(f, os[r].w, num.w);
+      }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint2 packed;
+    packed.x = pack_bf16x2(num.x * inv, num.y * inv);
+    packed.y = pack_bf16x2(num.z * inv, num.w * inv);
+    *reinterpret_cast<uint2*>(out + ((size_t)b * H + h) * kD + d4) = packed;
+  }
+  cluster_sync_all();   // no CTA leaves while its partial may still be read
+}
+
 // -------------------------------------------------------------- host side
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -974,6 +1596,124 @@ cslc_status run_decode_step(const cslc_decode_layer* layers, int n_layers, int B
   return CSLC_OK;
 }
 
+// ---- fused tail: one cluster of CL CTAs per sequence (CL a power of two <= 16)
+template <bool SPARSE, int CL>
+static cudaError_t launch_tail(const cslc_decode_layer& l, int B, int H, const float* scores, const DecodeWs& w,
+                               bool dependent, cudaStream_t stream) {
+  static int configured_for = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_for != dev) {
+    cudaFuncSetAttribute(decode_tail_kernel<SPARSE, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tail_smem_bytes(128));
+    if (CL > 8) cudaFuncSetAttribute(decode_tail_kernel<SPARSE, CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    configured_for = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, B);
+  cfg.blockDim = dim3(TAIL_THREADS);
+  cfg.dynamicSmemBytes = tail_smem_bytes(H);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = CL;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (dependent) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, decode_tail_kernel<SPARSE, CL>, l.q, l.nope, l.rope, l.kv_scale, l.n_entries,
+                            l.n_max, scores, (const uint32_t*)w.hist, w.cand, SPARSE ? l.topk : 0, H,
+                            l.scale * kLog2e, SPARSE ? l.idx_out : (int32_t*)nullptr, l.out);
+}
+
+template <bool SPARSE>
+static cudaError_t launch_tail_cl(int CL, const cslc_decode_layer& l, int B, int H, const float* scores,
+                                  const DecodeWs& w, bool dependent, cudaStream_t stream) {
+  switch (CL) {
+    case 1: return launch_tail<SPARSE, 1>(l, B, H, scores, w, dependent, stream);
+    case 2: return launch_tail<SPARSE, 2>(l, B, H, scores, w, dependent, stream);
+    case 4: return launch_tail<SPARSE, 4>(l, B, H, scores, w, dependent, stream);
+    case 8: return launch_tail<SPARSE, 8>(l, B, H, scores, w, dependent, stream);
+    default: return launch_tail<SPARSE, 16>(l, B, H, scores, w, dependent, stream);
+  }
+}
+
+// Per device, once: the SM count and whether 16-CTA clusters of the tail
+// kernel fit (a non-portable size).
+struct TailDevice {
+  int sms = 0;
+  bool cl16 = false;
+};
+static bool tail_device(TailDevice* out) {
+  constexpr int kMaxDevices = 64;
+  static TailDevice info[kMaxDevices];
+  static bool known[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (!known[dev]) {
+    TailDevice t;
+    if (cudaDeviceGetAttribute(&t.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    cudaFuncSetAttribute(decode_tail_kernel<true, 16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(decode_tail_kernel<true, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tail_smem_bytes(128));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1);
+    cfg.blockDim = dim3(TAIL_THREADS);
+    cfg.dynamicSmemBytes = tail_smem_bytes(128);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 16;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, decode_tail_kernel<true, 16>, &cfg);
+    if (e != cudaSuccess) cudaGetLastError();
+    t.cl16 = e == cudaSuccess && n > 0;
+    info[dev] = t;
+    known[dev] = true;
+  }
+  *out = info[dev];
+  return true;
+}
+
+// The tail of a CSA layer as one cluster launch when it fits: the cluster
+// size aims at one CTA per SM over the batch (a CTA of this kernel takes a
+// whole SM), and a cluster must cover the context with its bitmaps (131,072
+// entries per CTA). HCA layers keep the split attention + combine kernels.
+// Returns false to use the separate kernels.
+static bool run_tail_fused(const cslc_decode_layer& l, int B, int H, const float* scores, const DecodeWs& w,
+                           bool dependent, cudaStream_t stream, cslc_status* st) {
+  TailDevice dv;
+  if (!tail_device(&dv)) return false;
+  // a CTA takes a whole SM, so 16-CTA clusters only fit a few GPCs at a time:
+  // 16 only when a context needs it
+  const int cl_max = dv.cl16 ? 16 : 8;
+  int CL = 1;
+  while (CL < 8 && (long long)B * CL * 2 <= dv.sms) CL *= 2;
+  // small batches (B x 4 < SMs) keep the separate kernels: their clusters
+  // would hold whole SMs that the other layers' concurrent kernels need
+  // (measured: hybrid 1M step, B = 8, 189 us split vs 204 us fused; CSA
+  // 64 x 32,768, 120 us split vs 103 us fused)
+  if (l.kind != 0 || (long long)B * 4 < dv.sms) return false;
+  while (CL < cl_max && (long long)l.n_max > (long long)CL * TAIL_BM_WORDS * 32) CL *= 2;
+  if ((long long)l.n_max > (long long)CL * TAIL_BM_WORDS * 32) return false;
+  const cudaError_t e = launch_tail_cl<true>(CL, l, B, H, scores, w, dependent, stream);
+  *st = e == cudaSuccess ? CSLC_OK : set_error(CSLC_ERR_CUDA, "decode tail launch: %s", cudaGetErrorString(e));
+  return true;
+}
+
 static cslc_status run_layer(const cslc_decode_layer& l, int B, int H, int HI, DecodeWs& w, cudaStream_t stream) {
   {
     cslc_status st;
@@ -991,6 +1731,7 @@ static cslc_status run_layer(const cslc_decode_layer& l, int B, int H, int HI, D
         st = check_launch("decode_scores_kernel");
         if (st != CSLC_OK) return st;
       }
+      if (B > 0 && run_tail_fused(l, B, H, scores, w, l.n_max > 0, stream, &st)) return st;
       st = run_topk_stages(scores, l.n_entries, B, l.n_max, l.topk, w, idx, stream);
       if (st != CSLC_OK) return st;
       st = run_attention(l, B, H, idx, w, stream);

@@ -109,6 +109,43 @@ def test_decode_small_csa_and_hca_layers(C):
     assert_close(f64(lh.out), o_ref, rel=REL_L2_FP8, what="hca out")
 
 
+@pytest.mark.parametrize("H,n_max,want_scores,ties", [(64, 6000, True, False), (128, 5003, True, True),
+                                                     (16, 4100, False, False)])
+def test_decode_csa_large_batch(C, H, n_max, want_scores, ties):
+    """A batch large enough for the one-launch cluster tail (select, order,
+    attention and combine of a CSA layer, one cluster per sequence), with
+    contexts of 0, 1, fewer than k, exactly k, k + 1 and up to n_max entries
+    (n_max = 5003 takes the unvectorised score scan), tied scores from
+    duplicated keys, and the scores kept in the library's workspace."""
+    B, topk = 40, 1024
+    d = W.DecodeShape(B=B, H=H, kinds=("csa",), n_entries=(n_max,), topk=topk)
+    base = [0, 1, 300, topk, topk + 1, 2000, n_max - 1, n_max]
+    n_list = [base[b % len(base)] if b < 2 * len(base) else int(np.random.default_rng(b).integers(0, n_max + 1))
+              for b in range(B)]
+    x, n = _layer_inputs(d, 0, 47 + H, n_list)
+    if ties:
+        x["k_idx"][:, 100:400] = x["k_idx"][:, 0:300]
+    lc = _gpu_layer(C, d, "csa", x, n, topk, want_scores=want_scores)
+    C.decode_step([lc], HI=8)
+    torch.cuda.synchronize()
+    if want_scores:
+        _check_csa_layer(lc, x, n_list, topk, _oracle_kv(x))
+    else:
+        idx = lc.idx_out.cpu().numpy()
+        s_ref = O.decode_indexer_scores(f64(x["q_idx"]), f64(x["w"]), f64(x["k_idx"]), n_list)
+        kv_hat, out = _oracle_kv(x), f64(lc.out)
+        n_diff = 0
+        for b in range(B):
+            assert np.sum(idx[b] >= 0) == min(topk, n_list[b]) and np.all(idx[b][idx[b] >= 0] < n_list[b])
+            sel = idx[b][idx[b] >= 0]
+            assert np.all(np.diff(sel) > 0)
+            n_diff += not check_selection(idx[b], O.topk_select_row(s_ref[b], n_list[b], topk), s_ref[b],
+                                          n_list[b], topk)
+            o_ref, _ = O.attend(f64(x["q"])[b], kv_hat[b, sel], d.scale)
+            assert_close(out[b], O.round_bf16(o_ref), rel=REL_L2_FP8, what=f"csa out seq {b}")
+        assert n_diff <= max_differing(B), n_diff
+
+
 def test_decode_csa_topk_covering_everything_equals_dense(C):
     d = W.DecodeShape(B=2, H=16, kinds=("csa",), n_entries=(700,), topk=2048)
     n_list = [700, 650]
