@@ -70,7 +70,7 @@ __all__ = [
     "attend", "sparse_attention", "dense_causal_attention",
     "E4M3_MAX", "e4m3_decode", "e4m3_encode", "quantize_kv_mixed",
     "dequantize_kv_mixed", "decode_indexer_scores", "decode_csa_layer",
-    "decode_hca_layer", "project", "compressor_front_end",
+    "decode_hca_layer", "project", "compressor_front_end", "quantize_rows_e4m3", "indexer_scores_fp8",
 ]
 
 F64 = np.float64
@@ -387,6 +387,34 @@ def quantize_kv_mixed(e):
     scaled = (nope / scale[..., None]).astype(np.float32)
     codes = e4m3_encode(scaled.astype(F64))
     return codes, e[..., 64:].copy(), scale
+
+
+def quantize_rows_e4m3(x):
+    """Rows of x [..., d] as e4m3 codes with one fp32 scale per row ([EXPL]
+    §1.4: an FP8 form of the lightning indexer's operands). The rule is the
+    one of the mixed KV layout (reading R7): s = amax / 448 in fp32 (1 when the
+    row is zero), codes = RNE-saturate(x / s) with the division in fp32.
+    Returns (codes uint8 [..., d], scale float32 [...]).
+    """
+    x = np.asarray(x, dtype=F64).astype(np.float32)
+    amax = np.abs(x).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    scaled = (x / scale[..., None]).astype(np.float32)
+    return e4m3_encode(scaled.astype(F64)), scale
+
+
+def indexer_scores_fp8(q8, q_scale, w, k8, k_scale, m: int, q_pos0: int = 0, rows=None):
+    """Indexer scores from e4m3 operands ([EXPL] §1.4; formula of reading R4):
+    the scores of the values the codes stand for, q_I = decode(q8) * q_scale
+    per (token, head) row and k_I = decode(k8) * k_scale per entry, in float64,
+    rounded to fp32.
+
+    q8: [B, L, H_I, d_I] uint8, q_scale: [B, L, H_I]; w: [B, L, H_I];
+    k8: [B, N_c, d_I] uint8, k_scale: [B, N_c].
+    """
+    q = e4m3_decode(q8) * np.asarray(q_scale, dtype=F64)[..., None]
+    k = e4m3_decode(k8) * np.asarray(k_scale, dtype=F64)[..., None]
+    return indexer_scores(q, w, k, m, q_pos0, rows=rows)
 
 
 def dequantize_kv_mixed(nope_codes, rope, scale):

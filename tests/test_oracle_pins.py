@@ -463,6 +463,61 @@ def test_quantize_kv_mixed(O):
     assert np.all((top[mask] & 0x7F) == 0x7E)
 
 
+# ------------------------------------------------- FP8 indexer operands ---
+# (numpy oracle only: the FP8 indexer variant is not timed on the CPU, so the
+# C++ oracle does not carry it)
+
+def test_quantize_rows_e4m3_against_torch_cast():
+    N = NUMPY_ORACLE
+    x = bf16_values((5, 33, 64), std=3.0)
+    x[2, 4] = 0.0
+    codes, scale = N.quantize_rows_e4m3(x)
+    assert codes.shape == x.shape and codes.dtype == np.uint8 and scale.dtype == np.float32
+    xf = torch.from_numpy(x).float()
+    amax = xf.abs().amax(dim=-1)
+    s_ref = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))       # fp32 division
+    np.testing.assert_array_equal(scale, s_ref.numpy())
+    c_ref = (xf / s_ref[..., None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(codes, c_ref)
+    assert scale[2, 4] == 1.0 and np.all(codes[2, 4] == 0)
+    j = np.abs(x).argmax(axis=-1)
+    top = np.take_along_axis(codes, j[..., None], axis=-1)[..., 0]
+    assert np.all((top[np.abs(x).max(axis=-1) > 0] & 0x7F) == 0x7E)
+
+
+def test_indexer_scores_fp8_single_head_is_relu_gemm_of_torch_decoded_values():
+    N = NUMPY_ORACLE
+    B, L, n_c, m = 2, 24, 9, 2
+    q8, qs = N.quantize_rows_e4m3(bf16_values((B, L, 1, 64)))
+    k8, ks = N.quantize_rows_e4m3(bf16_values((B, n_c, 64)))
+    w = np.ones((B, L, 1))
+    got = N.indexer_scores_fp8(q8, qs, w, k8, ks, m)
+    qd = torch.from_numpy(q8).view(torch.float8_e4m3fn).double() * torch.from_numpy(qs).double()[..., None]
+    kd = torch.from_numpy(k8).view(torch.float8_e4m3fn).double() * torch.from_numpy(ks).double()[..., None]
+    ref = torch.relu(torch.matmul(qd[:, :, 0], kd.transpose(1, 2))).float().double().numpy()
+    for t in range(L):
+        nv = N.n_visible(t, m, n_c)
+        np.testing.assert_array_equal(got[:, t, :nv], ref[:, t, :nv])
+        assert np.all(got[:, t, nv:] == -np.inf)
+
+
+def test_indexer_scores_fp8_scale_equivariance_and_bf16_closeness():
+    N = NUMPY_ORACLE
+    B, L, HI, n_c, m = 1, 40, 4, 12, 3
+    q, k = bf16_values((B, L, HI, 64)), bf16_values((B, n_c, 64))
+    w = RNG.uniform(0, 1, (B, L, HI))
+    q8, qs = N.quantize_rows_e4m3(q)
+    k8, ks = N.quantize_rows_e4m3(k)
+    s1 = N.indexer_scores_fp8(q8, qs, w, k8, ks, m)
+    s2 = N.indexer_scores_fp8(q8, qs, w, k8, 2 * ks, m)
+    vis = np.isfinite(s1)
+    np.testing.assert_array_equal(s2[vis], 2 * s1[vis])       # power-of-two scale: exact
+    # within the e4m3 rounding of both operands of the bf16 path's scores
+    ref = N.indexer_scores(q, w, k, m)
+    bound = np.einsum("blh,blhd,bnd->bln", w, np.abs(q), np.abs(k)) * (2 * 2.0 ** -4 + 2.0 ** -8)
+    assert np.all(np.abs(s1[vis] - ref[vis]) <= bound[vis] + 1e-6)
+
+
 # ------------------------------------------------------------------ decode ---
 
 def test_decode_layers_reduce_to_dense_and_library(O):
