@@ -541,24 +541,32 @@ def measure(name, C, args, world, rank, local, peaks, flush, with_e2e=True, min_
     return res
 
 
-def measure_indexer_bf16(C, device, flush, reps=10):
-    """The indexer + top-k of the 65,536-token CSA workload with fp32 and with
-    bf16-stored scores (first page §1.4: scores FP32 -> BF16 for a faster
-    top-k): CUDA-event times (L2 flushed before each), and the recall of the
-    bf16 path's selection against the fp32 path's over every query row."""
+def measure_indexer_variants(C, device, flush, reps=10):
+    """The indexer + top-k of the 65,536-token CSA workload in its three forms
+    (first page §1.4: a low-precision indexer): fp32 scores from bf16
+    operands (the headline path), bf16-stored scores, and e4m3 operands with
+    per-row scales (fp32 scores). CUDA-event medians with L2 flushed before
+    each call; the e4m3 rows are quantised beforehand (their quantisation is
+    timed on its own), and the recall of each variant's selection against the
+    fp32 path's over every query row."""
     wl = W.WORKLOADS["csa_prefill"]
     s = wl.csa
     x = W.prefill_inputs(s, wl.wid, device=device)
     idx32 = torch.empty(s.B, s.L, s.topk, dtype=torch.int32, device=device)
     idx16 = torch.empty_like(idx32)
+    idx8 = torch.empty_like(idx32)
     ws32 = torch.empty(max(16, C.indexer_topk_workspace_bytes(s.B, s.L, s.n_c, s.HI, s.topk)), dtype=torch.uint8,
                        device=device)
     ws16 = torch.empty(max(16, C.indexer_topk_bf16_workspace_bytes(s.B, s.L, s.n_c, s.HI, s.topk)), dtype=torch.uint8,
                        device=device)
+    q8, qs = C.quantize_rows_e4m3(x["q_idx"])
+    k8, ks = C.quantize_rows_e4m3(x["k_idx"])
     run32 = lambda: C.csa_indexer_topk(x["q_idx"], x["w"], x["k_idx"], m=s.m, topk=s.topk, idx=idx32, ws=ws32)
     run16 = lambda: C.csa_indexer_topk_bf16(x["q_idx"], x["w"], x["k_idx"], m=s.m, topk=s.topk, idx=idx16, ws=ws16)
+    run8 = lambda: C.csa_indexer_topk_fp8(q8, qs, x["w"], k8, ks, m=s.m, topk=s.topk, idx=idx8, ws=ws32)
+    quant = lambda: (C.quantize_rows_e4m3(x["q_idx"], q8, qs), C.quantize_rows_e4m3(x["k_idx"], k8, ks))
     out = {}
-    for name, fn in (("fp32", run32), ("bf16", run16)):
+    for name, fn in (("fp32", run32), ("bf16_scores", run16), ("fp8_operands", run8), ("fp8_quantize", quant)):
         for _ in range(3):
             fn()
         ts = []
@@ -571,19 +579,20 @@ def measure_indexer_bf16(C, device, flush, reps=10):
             torch.cuda.synchronize()
             ts.append(a_.elapsed_time(b_))
         out[f"ms_{name}"] = sorted(ts)[len(ts) // 2]
-    # recall: |sel_fp32 & sel_bf16| / |sel_fp32| over all rows (selections are ascending, -1 padded)
-    kept = 0
-    for r0 in range(0, s.L, 4096):
-        a_ = idx32[0, r0:r0 + 4096].long()
-        b_ = idx16[0, r0:r0 + 4096].long()
-        big = s.n_c + 1
-        a_ = torch.where(a_ < 0, torch.full_like(a_, big), a_)
-        b_ = torch.where(b_ < 0, torch.full_like(b_, -1), b_)
-        pos = torch.searchsorted(b_.contiguous(), a_.contiguous()).clamp(max=s.topk - 1)
-        kept += int((torch.gather(b_, 1, pos) == a_).sum())
-    total = int((idx32 >= 0).sum())
-    out["recall_vs_fp32"] = kept / max(1, total)
-    out["speedup"] = out["ms_fp32"] / out["ms_bf16"]
+
+    def recall(idx):   # |sel_fp32 & sel| / |sel_fp32| over all rows (selections ascending, -1 padded)
+        kept = 0
+        for r0 in range(0, s.L, 4096):
+            a_ = idx32[0, r0:r0 + 4096].long()
+            b_ = idx[0, r0:r0 + 4096].long()
+            a_ = torch.where(a_ < 0, torch.full_like(a_, s.n_c + 1), a_)
+            b_ = torch.where(b_ < 0, torch.full_like(b_, -1), b_)
+            pos = torch.searchsorted(b_.contiguous(), a_.contiguous()).clamp(max=s.topk - 1)
+            kept += int((torch.gather(b_, 1, pos) == a_).sum())
+        return kept / max(1, int((idx32 >= 0).sum()))
+
+    out["recall_bf16_scores_vs_fp32"] = recall(idx16)
+    out["recall_fp8_operands_vs_fp32"] = recall(idx8)
     out["workload"] = "indexer + top-k of csa_prefill (L=65536, 16384 entries, 8 x 64, top-k 1024)"
     return out
 
@@ -889,7 +898,7 @@ def main():
             secondary[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "kernel_ms", "roofline",
                                                   "clocks", "config", "steps")}
             secondary[name]["gpu_launches"] = r["gpu_launches"]
-        secondary["indexer_topk_bf16_scores"] = measure_indexer_bf16(C, torch.device("cuda", local), flush)
+        secondary["indexer_topk_variants"] = measure_indexer_variants(C, torch.device("cuda", local), flush)
 
     cpu = None
     if rank == 0 and world == 1:

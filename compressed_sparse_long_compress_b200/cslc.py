@@ -30,7 +30,7 @@ ABI_SYMBOLS = [
     "cslc_decode_topk_workspace_bytes", "cslc_decode_topk", "cslc_decode_topk_noalloc", "cslc_decode_append",
     "csa_compress_front_end", "hca_compress_front_end",
     "csa_indexer_topk_bf16_workspace_bytes", "csa_indexer_topk_bf16", "csa_topk_bf16",
-    "cslc_testing_set_wait_limits",
+    "cslc_testing_set_wait_limits", "cslc_quantize_rows_e4m3", "csa_indexer_topk_fp8",
 ]
 
 
@@ -81,6 +81,9 @@ def _load():
                                           P, P, P, c_size_t, P]),
         "csa_topk_bf16": (c_int, [P, c_int, c_int, c_int, c_int, c_int, c_int, P, P]),
         "cslc_testing_set_wait_limits": (c_int, [ctypes.c_uint64, ctypes.c_uint32]),
+        "cslc_quantize_rows_e4m3": (c_int, [P, ctypes.c_int64, c_int, P, P, P]),
+        "csa_indexer_topk_fp8": (c_int, [P, P, P, P, P, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                         P, P, P, c_size_t, P]),
         "hca_compress_front_end": (c_int, [P, P, P, c_int, c_int, c_int, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -230,6 +233,46 @@ def csa_indexer_topk_bf16(q_idx, w, k_idx, m: int, topk: int, q_pos0: int = 0, s
     _check(LIB.csa_indexer_topk_bf16(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, L, Nc, HI, dI, m, q_pos0, topk,
                                      _ptr(scores), _ptr(idx), _ptr(ws) if nbytes else None,
                                      ws.numel() if (nbytes and ws is not None) else 0, _stream(stream)))
+    return idx, scores
+
+
+def quantize_rows_e4m3(x, codes=None, scales=None, stream=None):
+    """Rows x [..., 64] bf16 -> (codes uint8 [..., 64], scales fp32 [...])."""
+    _need(x, BF16, "x")
+    if x.shape[-1] != 64:
+        raise ValueError("quantize_rows_e4m3: rows of 64 values")
+    rows = x.numel() // 64
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=U8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=F32, device=x.device)
+    _need(codes, U8, "codes", tuple(x.shape)); _need(scales, F32, "scales", tuple(x.shape[:-1]))
+    _check(LIB.cslc_quantize_rows_e4m3(_ptr(x), rows, 64, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def csa_indexer_topk_fp8(q8, q_scale, w, k8, k_scale, m: int, topk: int, q_pos0: int = 0, scores=None, idx=None,
+                         ws=None, stream=None):
+    """csa_indexer_topk on e4m3 operands (codes + per-row scales from
+    quantize_rows_e4m3). Returns (idx, scores or None); scores=True allocates
+    a [B, L, Nc] fp32 tensor."""
+    B, L, HI, dI = q8.shape
+    Nc = k8.shape[1]
+    _need(q8, U8, "q8"); _need(q_scale, F32, "q_scale", (B, L, HI)); _need(w, BF16, "w", (B, L, HI))
+    _need(k8, U8, "k8", (B, Nc, dI)); _need(k_scale, F32, "k_scale", (B, Nc))
+    if scores is True:
+        scores = torch.empty(B, L, Nc, dtype=F32, device=q8.device)
+    if scores is not None:
+        _need(scores, F32, "scores", (B, L, Nc))
+    if idx is None:
+        idx = torch.empty(B, L, topk, dtype=I32, device=q8.device)
+    _need(idx, I32, "idx", (B, L, topk))
+    nbytes = LIB.csa_indexer_topk_workspace_bytes(B, L, Nc, HI, topk, int(scores is not None))
+    if nbytes and (ws is None or ws.numel() < nbytes):
+        ws = torch.empty(nbytes, dtype=U8, device=q8.device)
+    _check(LIB.csa_indexer_topk_fp8(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), B, L, Nc, HI, dI, m,
+                                    q_pos0, topk, _ptr(scores), _ptr(idx), _ptr(ws) if nbytes else None,
+                                    ws.numel() if (nbytes and ws is not None) else 0, _stream(stream)))
     return idx, scores
 
 

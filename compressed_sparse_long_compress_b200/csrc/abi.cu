@@ -31,6 +31,9 @@ cslc_status launch_decode_append(const uint16_t*, const uint16_t*, const uint16_
                                  const uint16_t*, const int32_t*, int, int, int, uint16_t*, uint16_t*, uint16_t*,
                                  uint16_t*, uint8_t*, uint16_t*, float*, uint16_t*, int, int32_t*, cudaStream_t);
 cslc_status launch_quantize_kv(const uint16_t*, long long, uint8_t*, uint16_t*, float*, cudaStream_t);
+cslc_status launch_quantize_rows64(const uint16_t*, long long, uint8_t*, float*, cudaStream_t);
+cslc_status launch_indexer_scores_fp8(const uint8_t*, const float*, const uint16_t*, const uint8_t*, const float*, int,
+                                      int, int, int, int, int, int, int, float*, int, cudaStream_t);
 cslc_status launch_indexer_scores(const uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int,
                                   int, int, int, int, void*, bool, int, cudaStream_t);
 cslc_status launch_topk_rows(const void*, bool, int, int, int, int, int, int, int, int, int, int32_t*,
@@ -210,20 +213,51 @@ static size_t indexer_ws_bytes(int B, int L, int Nc, int score_bytes, int scores
   return (size_t)n_buf * B * R * Nc * score_bytes;
 }
 
+// The indexer's operands: bf16 q_I / k_I, or e4m3 codes with per-row scales.
+struct IndexerOperands {
+  const void* q;
+  const cslc_bf16* w;
+  const void* k;
+  const float* q_scale;
+  const float* k_scale;
+  bool fp8;
+};
+
+// Scores of rows [r0, r1) into buf ([B][R][Nc]; fp32, or bf16 when bf16).
+static cslc_status launch_scores(const IndexerOperands& op, int B, int L, int Nc, int HI, int m, int q_pos0, int r0,
+                                 int r1, void* buf, bool bf16, int R, cudaStream_t stream) {
+  if (op.fp8)
+    return launch_indexer_scores_fp8(static_cast<const uint8_t*>(op.q), op.q_scale, op.w,
+                                     static_cast<const uint8_t*>(op.k), op.k_scale, B, L, Nc, HI, m, q_pos0, r0, r1,
+                                     static_cast<float*>(buf), R, stream);
+  return launch_indexer_scores(static_cast<const uint16_t*>(op.q), op.w, static_cast<const uint16_t*>(op.k), B, L,
+                               Nc, HI, m, q_pos0, r0, r1, buf, bf16, R, stream);
+}
+
 // The indexer and the top-k, with fp32 or bf16 scores (bf16: each fp32 score
 // rounded to nearest even before it is stored and selected on).
-static cslc_status indexer_topk_impl(const char* fn, const cslc_bf16* q_idx, const cslc_bf16* w,
-                                     const cslc_bf16* k_idx, int B, int L, int Nc, int HI, int dI, int m,
-                                     int q_pos0, int topk, void* scores, bool bf16, int32_t* idx, void* ws,
+static cslc_status indexer_topk_impl(const char* fn, const IndexerOperands& op, int B, int L, int Nc, int HI, int dI,
+                                     int m, int q_pos0, int topk, void* scores, bool bf16, int32_t* idx, void* ws,
                                      size_t ws_bytes, cudaStream_t stream) {
   REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE, "%s: negative size / m < 1", fn);
   REQUIRE(dI == kDI, CSLC_ERR_UNSUPPORTED, "%s: d_I must be 64 (got %d)", fn, dI);
   REQUIRE(HI >= 1 && HI <= 16, CSLC_ERR_UNSUPPORTED, "%s: H_I must be in [1, 16]", fn);
+  REQUIRE(!op.fp8 || is_pow2(HI), CSLC_ERR_UNSUPPORTED, "%s: H_I must be 1, 2, 4, 8 or 16 (got %d)", fn, HI);
   REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "%s: topk must be in [1, 2048]", fn);
   REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "%s: Nc must be <= %d", fn, kMaxPrefillTopkNc);
   if ((long long)B * L == 0) return CSLC_OK;
   REQUIRE_PTR(idx);
-  if (Nc > 0) { REQUIRE_PTR(q_idx); REQUIRE_PTR(w); REQUIRE_PTR(k_idx); }
+  if (Nc > 0) {
+    const void* q_idx = op.q;
+    const void* k_idx = op.k;
+    const cslc_bf16* w = op.w;
+    REQUIRE_PTR(q_idx); REQUIRE_PTR(w); REQUIRE_PTR(k_idx);
+    if (op.fp8) {
+      const float* q_scale = op.q_scale;
+      const float* k_scale = op.k_scale;
+      REQUIRE_PTR(q_scale); REQUIRE_PTR(k_scale);
+    }
+  }
   if (scores) REQUIRE_PTR(scores);
   const int sb = bf16 ? 2 : 4;
   const size_t need = indexer_ws_bytes(B, L, Nc, sb, scores != nullptr);
@@ -233,7 +267,7 @@ static cslc_status indexer_topk_impl(const char* fn, const cslc_bf16* q_idx, con
   }
   cslc_status st;
   if (scores) {
-    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, scores, bf16, L, stream);
+    st = launch_scores(op, B, L, Nc, HI, m, q_pos0, 0, L, scores, bf16, L, stream);
     if (st != CSLC_OK) return st;
     return launch_topk_rows(scores, bf16, L, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
   }
@@ -242,7 +276,7 @@ static cslc_status indexer_topk_impl(const char* fn, const cslc_bf16* q_idx, con
   uint8_t* buf = static_cast<uint8_t*>(ws);
   if (L <= R || Nc == 0) {
     if (Nc > 0) {
-      st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, 0, L, buf, bf16, R, stream);
+      st = launch_scores(op, B, L, Nc, HI, m, q_pos0, 0, L, buf, bf16, R, stream);
       if (st != CSLC_OK) return st;
     }
     return launch_topk_rows(buf, bf16, R, 0, L, B, L, Nc, m, q_pos0, topk, idx, stream);
@@ -258,7 +292,7 @@ static cslc_status indexer_topk_impl(const char* fn, const cslc_bf16* q_idx, con
     uint8_t* bj = buf + j * block_bytes;
     cudaError_t e = i >= 2 ? cudaStreamWaitEvent(stream, o->freed[j], 0) : cudaSuccess;
     if (e != cudaSuccess) return set_error(CSLC_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
-    st = launch_indexer_scores(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, r0, r1, bj, bf16, R, stream);
+    st = launch_scores(op, B, L, Nc, HI, m, q_pos0, r0, r1, bj, bf16, R, stream);
     if (st != CSLC_OK) return st;
     e = cudaEventRecord(o->ready[j], stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(o->aux, o->ready[j], 0);
@@ -294,8 +328,9 @@ size_t csa_indexer_topk_workspace_bytes(int B, int L, int Nc, int HI, int topk, 
 cslc_status csa_indexer_topk(const cslc_bf16* q_idx, const cslc_bf16* w, const cslc_bf16* k_idx, int B,
                              int L, int Nc, int HI, int dI, int m, int q_pos0, int topk, float* scores,
                              int32_t* idx, void* ws, size_t ws_bytes, cslc_stream_t stream) {
-  return indexer_topk_impl("csa_indexer_topk", q_idx, w, k_idx, B, L, Nc, HI, dI, m, q_pos0, topk, scores, false,
-                           idx, ws, ws_bytes, stream);
+  const IndexerOperands op{q_idx, w, k_idx, nullptr, nullptr, false};
+  return indexer_topk_impl("csa_indexer_topk", op, B, L, Nc, HI, dI, m, q_pos0, topk, scores, false, idx, ws, ws_bytes,
+                           stream);
 }
 
 size_t csa_indexer_topk_bf16_workspace_bytes(int B, int L, int Nc, int HI, int topk, int scores_given) {
@@ -306,8 +341,28 @@ size_t csa_indexer_topk_bf16_workspace_bytes(int B, int L, int Nc, int HI, int t
 cslc_status csa_indexer_topk_bf16(const cslc_bf16* q_idx, const cslc_bf16* w, const cslc_bf16* k_idx, int B,
                                   int L, int Nc, int HI, int dI, int m, int q_pos0, int topk, cslc_bf16* scores,
                                   int32_t* idx, void* ws, size_t ws_bytes, cslc_stream_t stream) {
-  return indexer_topk_impl("csa_indexer_topk_bf16", q_idx, w, k_idx, B, L, Nc, HI, dI, m, q_pos0, topk, scores,
-                           true, idx, ws, ws_bytes, stream);
+  const IndexerOperands op{q_idx, w, k_idx, nullptr, nullptr, false};
+  return indexer_topk_impl("csa_indexer_topk_bf16", op, B, L, Nc, HI, dI, m, q_pos0, topk, scores, true, idx, ws,
+                           ws_bytes, stream);
+}
+
+cslc_status csa_indexer_topk_fp8(const uint8_t* q8, const float* q_scale, const cslc_bf16* w, const uint8_t* k8,
+                                 const float* k_scale, int B, int L, int Nc, int HI, int dI, int m, int q_pos0,
+                                 int topk, float* scores, int32_t* idx, void* ws, size_t ws_bytes,
+                                 cslc_stream_t stream) {
+  const IndexerOperands op{q8, w, k8, q_scale, k_scale, true};
+  return indexer_topk_impl("csa_indexer_topk_fp8", op, B, L, Nc, HI, dI, m, q_pos0, topk, scores, false, idx, ws,
+                           ws_bytes, stream);
+}
+
+cslc_status cslc_quantize_rows_e4m3(const cslc_bf16* x, int64_t rows, int d, uint8_t* codes, float* scales,
+                                    cslc_stream_t stream) {
+  REQUIRE(rows >= 0, CSLC_ERR_SHAPE, "cslc_quantize_rows_e4m3: negative size");
+  REQUIRE(d == 64, CSLC_ERR_UNSUPPORTED, "cslc_quantize_rows_e4m3: d must be 64 (got %d)", d);
+  REQUIRE(rows <= (1ll << 34), CSLC_ERR_UNSUPPORTED, "cslc_quantize_rows_e4m3: at most 2^34 rows");
+  if (rows == 0) return CSLC_OK;
+  REQUIRE_PTR(x); REQUIRE_PTR(codes); REQUIRE_PTR(scales);
+  return launch_quantize_rows64(x, rows, codes, scales, stream);
 }
 
 cslc_status csa_topk(const float* scores, int B, int L, int Nc, int m, int q_pos0, int topk, int32_t* idx,

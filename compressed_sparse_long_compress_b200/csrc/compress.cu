@@ -142,16 +142,24 @@ cslc_status launch_compress(const uint16_t* c, const uint16_t* z, const uint16_t
 // One entry's row (lane l holds dims 2l, 2l+1 in `lo` and 64+2l, 64+2l+1 in
 // `hi`) into the mixed layout; shared by the bulk quantiser and the decode
 // append so that both produce identical codes.
-__device__ __forceinline__ void quantize_row(uint32_t lo, uint32_t hi, int lane, uint8_t* __restrict__ nope_row,
-                                             uint16_t* __restrict__ rope_row, float* __restrict__ scale_out) {
+// 64 bf16 values (lane l holds 2l, 2l+1 in `lo`) as e4m3 codes with one fp32
+// scale: s = amax / 448 (1 for a zero row), codes = RNE-saturate(x / s), the
+// division in fp32.
+__device__ __forceinline__ void e4m3_row64(uint32_t lo, int lane, uint8_t* __restrict__ codes_row,
+                                           float* __restrict__ scale_out) {
   const float x0 = bf16_lo(lo), x1 = bf16_hi(lo);
   const float amax = warp_max(fmaxf(fabsf(x0), fabsf(x1)));
   const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
   const float2 q = make_float2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
   const __nv_fp8x2_storage_t codes = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
-  reinterpret_cast<uint16_t*>(nope_row)[lane] = codes;
-  reinterpret_cast<uint32_t*>(rope_row)[lane] = hi;
+  reinterpret_cast<uint16_t*>(codes_row)[lane] = codes;
   if (lane == 0) *scale_out = s;
+}
+
+__device__ __forceinline__ void quantize_row(uint32_t lo, uint32_t hi, int lane, uint8_t* __restrict__ nope_row,
+                                             uint16_t* __restrict__ rope_row, float* __restrict__ scale_out) {
+  e4m3_row64(lo, lane, nope_row, scale_out);
+  reinterpret_cast<uint32_t*>(rope_row)[lane] = hi;
 }
 
 __global__ void __launch_bounds__(256) quantize_kv_kernel(const uint16_t* __restrict__ kv,
@@ -164,6 +172,24 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(const uint16_t* __rest
   if (e >= n_entries) return;
   const uint32_t* row = reinterpret_cast<const uint32_t*>(kv + e * kD);
   quantize_row(row[lane], row[32 + lane], lane, nope + e * kNope, rope + e * kRope, scale + e);
+}
+
+// Rows of 64 values (the indexer's q_I / k_I rows) as e4m3 codes + a scale each.
+__global__ void __launch_bounds__(256) quantize_rows64_kernel(const uint16_t* __restrict__ x, long long rows,
+                                                              uint8_t* __restrict__ codes,
+                                                              float* __restrict__ scales) {
+  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  e4m3_row64(reinterpret_cast<const uint32_t*>(x + r * 64)[lane], lane, codes + r * 64, scales + r);
+}
+
+cslc_status launch_quantize_rows64(const uint16_t* x, long long rows, uint8_t* codes, float* scales,
+                                   cudaStream_t stream) {
+  if (rows == 0) return CSLC_OK;
+  const long long blocks = (rows * 32 + 255) / 256;
+  quantize_rows64_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, rows, codes, scales);
+  return check_launch("quantize_rows64_kernel");
 }
 
 cslc_status launch_quantize_kv(const uint16_t* kv, long long n, uint8_t* nope, uint16_t* rope,

@@ -180,6 +180,59 @@ cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const
                                  int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
                                  void* scores, bool bf16_out, int rows_in_buf, cudaStream_t stream);
 
+cslc_status launch_indexer_sm100_fp8(const uint8_t* q8, const float* q_scale, const uint16_t* w, const uint8_t* k8,
+                                     const float* k_scale, int B, int L, int Nc, int HI, int m, int q_pos0,
+                                     int row_begin, int row_end, float* scores, int rows_in_buf, cudaStream_t stream);
+
+// FP8 operands on the CUDA cores, for inputs smaller than one tensor-core
+// tile (fewer than 256 (token, head) rows or 128 entries): one thread per
+// (row, entry), the code products summed in fp32 and the scales applied as
+// the tensor-core kernel applies them.
+__global__ void __launch_bounds__(256) indexer_fp8_small_kernel(
+    const uint8_t* __restrict__ q8, const float* __restrict__ q_scale, const uint16_t* __restrict__ w,
+    const uint8_t* __restrict__ k8, const float* __restrict__ k_scale, int B, int L, int Nc, int HI, int m,
+    int q_pos0, int row_begin, int row_end, float* __restrict__ scores, int rows_in_buf) {
+  const int R = row_end - row_begin;
+  const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (long long)B * R * Nc) return;
+  const int i = (int)(id % Nc);
+  const long long br = id / Nc;
+  const int r = (int)(br % R), b = (int)(br / R);
+  const int t = row_begin + r;
+  if (i >= n_visible((long long)q_pos0 + t, m, Nc)) return;
+  const uint16_t* kr = reinterpret_cast<const uint16_t*>(k8 + ((size_t)b * Nc + i) * 64);
+  float acc = 0.f;
+  for (int h = 0; h < HI; ++h) {
+    const size_t p = ((size_t)b * L + t) * HI + h;
+    const uint16_t* qr = reinterpret_cast<const uint16_t*>(q8 + p * 64);
+    float dot = 0.f;
+    for (int d = 0; d < 32; ++d) {
+      const __half2_raw qh = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)qr[d], __NV_E4M3);
+      const __half2_raw kh = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)kr[d], __NV_E4M3);
+      const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qh));
+      const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kh));
+      dot = fmaf(qf.x, kf.x, dot);
+      dot = fmaf(qf.y, kf.y, dot);
+    }
+    acc = fmaf(bf16_to_f(w[p]) * q_scale[p], fmaxf(dot, 0.f), acc);
+  }
+  scores[((size_t)b * rows_in_buf + r) * Nc + i] = k_scale[(size_t)b * Nc + i] * acc;
+}
+
+cslc_status launch_indexer_scores_fp8(const uint8_t* q8, const float* q_scale, const uint16_t* w, const uint8_t* k8,
+                                      const float* k_scale, int B, int L, int Nc, int HI, int m, int q_pos0,
+                                      int row_begin, int row_end, float* scores, int rows_in_buf,
+                                      cudaStream_t stream) {
+  if (row_end <= row_begin || B == 0 || Nc == 0) return CSLC_OK;
+  if ((long long)B * L * HI >= 256 && (long long)B * Nc >= 128)
+    return launch_indexer_sm100_fp8(q8, q_scale, w, k8, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores,
+                                    rows_in_buf, stream);
+  const long long n = (long long)B * (row_end - row_begin) * Nc;
+  indexer_fp8_small_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+      q8, q_scale, w, k8, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, rows_in_buf);
+  return check_launch("indexer_fp8_small_kernel");
+}
+
 // scores: fp32 [rows][Nc], or bf16 when bf16_out
 cslc_status launch_indexer_scores(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
                                   int B, int L, int Nc, int HI, int m, int q_pos0, int row_begin,

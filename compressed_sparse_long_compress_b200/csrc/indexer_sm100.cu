@@ -25,6 +25,14 @@
 //              stores those of visible entries.
 // TMEM: two accumulators of 256 columns (tile j+1 is computed while tile j is
 // read out). All waits are time-bounded (abort + device error word).
+//
+// FP8 variant (first page §1.4: a low-precision lightning indexer): q_I and
+// k_I arrive as e4m3 codes with one fp32 scale per (token, head) row and per
+// entry. The tiles are 64-byte rows in the 64-byte swizzle, the products are
+// kind::f8f6f4 (K = 32, two per tile) with fp32 accumulation, and since the
+// scales are positive, S[t, i] = k_scale[i] * sum_h (w[t, h] q_scale[t, h]) *
+// max(0, q8[t, h] . k8[i]): the producer folds q_scale into the head weights
+// and the epilogue multiplies by k_scale.
 
 #include "sm100.cuh"
 
@@ -77,12 +85,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void store_score(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_score(uint16_t* p, float v) { *p = __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
-template <int HI, typename OutT>
+template <int HI, typename OutT, bool FP8>
 __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
-    const uint16_t* __restrict__ w, int B, int L, int Nc, int m, int q_pos0, int row_begin, int row_end,
-    OutT* __restrict__ scores, int rows_in_buf, const __grid_constant__ CUtensorMap tm_q,
-    const __grid_constant__ CUtensorMap tm_k) {
+    const uint16_t* __restrict__ w, const float* __restrict__ q_scale, const float* __restrict__ k_scale, int B,
+    int L, int Nc, int m, int q_pos0, int row_begin, int row_end, OutT* __restrict__ scores, int rows_in_buf,
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
   constexpr int RT = IX_NP / HI;                 // query rows per tile
+  // bytes of a loaded tile (the shared-memory slots are sized for bf16)
+  constexpr uint32_t Q_TX = FP8 ? IX_NP * 64 : IX_Q_BYTES, K_TX = FP8 ? IX_ET * 64 : IX_K_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;                                        // [2][256 pairs][128 B]
@@ -156,13 +166,15 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
 #pragma unroll
       for (int x = 0; x < IX_NP / 32; ++x) {
         const long long p = p0 + x * 32 + lane;
-        w_s[qs * IX_NP + x * 32 + lane] = p < n_pairs ? bf16_to_f(w[p]) : 0.f;
+        float wv = p < n_pairs ? bf16_to_f(w[p]) : 0.f;
+        if constexpr (FP8) wv *= p < n_pairs ? q_scale[p] : 0.f;
+        w_s[qs * IX_NP + x * 32 + lane] = wv;
       }
       for (int r = lane; r < RT; r += 32)
         nv_s[qs * IX_NP + r] = t0 + r < row_end ? n_visible((long long)q_pos0 + t0 + r, m, Nc) : 0;
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars.q_full[qs], IX_Q_BYTES);
+        mbar_arrive_expect_tx(&bars.q_full[qs], Q_TX);
         tma_load_2d(q_s + qs * IX_Q_BYTES, &tm_q, 0, (int)p0, &bars.q_full[qs]);
         for (int et = et0; et < et0 + n_et; ++et, ++kt) {
           const int ks = kt % IX_KSTAGES;
@@ -171,7 +183,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bars.k_full[ks], IX_K_BYTES);
+          mbar_arrive_expect_tx(&bars.k_full[ks], K_TX);
           tma_load_2d(k_s + ks * IX_K_BYTES, &tm_k, 0, b * Nc + et * IX_ET, &bars.k_full[ks]);
         }
       }
@@ -188,7 +200,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
   } else if (warp == IX_MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t ID = idesc_bf16(IX_ET, IX_NP, false, false);
+      constexpr uint32_t ID = FP8 ? idesc_e4m3(IX_ET, IX_NP) : idesc_bf16(IX_ET, IX_NP, false, false);
       int rq = 0, kt = 0;
       bool ok = true;
       int b, t0, et0, n_et;
@@ -206,10 +218,17 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
           }
           tc_fence_after();
           const uint32_t k0 = smem_u32(k_s + ks * IX_K_BYTES);
+          if constexpr (FP8) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + ds * IX_NP, smem_desc_sw128(k0 + k * 32, 16, 1024),
-                     smem_desc_sw128(q0 + k * 32, 16, 1024), ID, k > 0 ? 1u : 0u);
+            for (int k = 0; k < 2; ++k)   // K = 32 e4m3 per product: 32 bytes along the 64-byte rows
+              mma_e4m3(tmem + ds * IX_NP, smem_desc_sw64(k0 + k * 32, 16, 512),
+                       smem_desc_sw64(q0 + k * 32, 16, 512), ID, k > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16(tmem + ds * IX_NP, smem_desc_sw128(k0 + k * 32, 16, 1024),
+                       smem_desc_sw128(q0 + k * 32, 16, 1024), ID, k > 0 ? 1u : 0u);
+          }
           mma_commit(&bars.k_empty[ks]);
           mma_commit(&bars.d_full[ds]);
         }
@@ -247,6 +266,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
         if (!__shfl_sync(0xffffffffu, (int)d_ok, 0)) { ok = false; break; }
         tc_fence_after();
         const int e = et * IX_ET + quad * 32 + lane;
+        float ksc = 1.f;
+        if constexpr (FP8) ksc = e < Nc ? k_scale[(size_t)b * Nc + e] : 0.f;
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ds * IX_NP + part * IX_EPI_COLS;
         // one 32-column chunk per TMEM wait; each score's head sum runs as two
         // independent FMA chains
@@ -276,7 +297,11 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
                 if (q & 1) s1 = fmaf(wq[q], x, s1); else s0 = fmaf(wq[q], x, s0);
               }
             }
-            if (e < nvr[r]) store_score(out0 + (size_t)r * Nc + e, s0 + s1);
+            if constexpr (FP8) {
+              if (e < nvr[r]) store_score(out0 + (size_t)r * Nc + e, ksc * (s0 + s1));
+            } else {
+              if (e < nvr[r]) store_score(out0 + (size_t)r * Nc + e, s0 + s1);
+            }
           }
         }
         tc_fence_before();
@@ -298,10 +323,11 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
 
 bool indexer_sm100_supported(int HI) { return HI == 1 || HI == 2 || HI == 4 || HI == 8 || HI == 16; }
 
-template <typename OutT>
-static cslc_status launch_indexer_sm100_t(const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int B,
-                                          int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
-                                          OutT* scores, int rows_in_buf, cudaStream_t stream) {
+template <typename OutT, bool FP8>
+static cslc_status launch_indexer_sm100_t(const void* q_idx, const uint16_t* w, const void* k_idx,
+                                          const float* q_scale, const float* k_scale, int B, int L, int Nc, int HI,
+                                          int m, int q_pos0, int row_begin, int row_end, OutT* scores,
+                                          int rows_in_buf, cudaStream_t stream) {
   static int configured_for = -1;
   static int n_sm = 148;
   int dev = 0;
@@ -309,11 +335,11 @@ static cslc_status launch_indexer_sm100_t(const uint16_t* q_idx, const uint16_t*
   const size_t smem = 1024 + 2 * IX_Q_BYTES + IX_KSTAGES * IX_K_BYTES + 2 * IX_NP * (sizeof(float) + sizeof(int)) +
                       sizeof(IxSmall);
   if (configured_for != dev) {
-    cudaFuncSetAttribute(indexer_sm100_kernel<1, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<2, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<4, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<8, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(indexer_sm100_kernel<16, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<1, OutT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<2, OutT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<4, OutT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<8, OutT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(indexer_sm100_kernel<16, OutT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     configured_for = dev;
   }
@@ -323,15 +349,18 @@ static cslc_status launch_indexer_sm100_t(const uint16_t* q_idx, const uint16_t*
   const int n_items = B * ((row_end - row_begin + RT - 1) / RT) * n_ch;
   const int grid = n_items < n_sm ? n_items : n_sm;
   CUtensorMap tm_q, tm_k;
-  if (!make_tmap_bf16_2d(&tm_q, q_idx, (uint64_t)B * L * HI, kDI, kDI * 2, IX_NP, 64) ||
-      !make_tmap_bf16_2d(&tm_k, k_idx, (uint64_t)B * Nc, kDI, kDI * 2, IX_ET, 64))
-    return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: tensor map encoding failed");
+  const bool maps_ok =
+      FP8 ? make_tmap_u8_rows64(&tm_q, q_idx, (uint64_t)B * L * HI, IX_NP) &&
+                make_tmap_u8_rows64(&tm_k, k_idx, (uint64_t)B * Nc, IX_ET)
+          : make_tmap_bf16_2d(&tm_q, q_idx, (uint64_t)B * L * HI, kDI, kDI * 2, IX_NP, 64) &&
+                make_tmap_bf16_2d(&tm_k, k_idx, (uint64_t)B * Nc, kDI, kDI * 2, IX_ET, 64);
+  if (!maps_ok) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: tensor map encoding failed");
   switch (HI) {
-    case 1: indexer_sm100_kernel<1, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 2: indexer_sm100_kernel<2, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 4: indexer_sm100_kernel<4, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 8: indexer_sm100_kernel<8, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    default: indexer_sm100_kernel<16, OutT><<<grid, IX_THREADS, smem, stream>>>(w, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 1: indexer_sm100_kernel<1, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 2: indexer_sm100_kernel<2, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 4: indexer_sm100_kernel<4, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 8: indexer_sm100_kernel<8, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    default: indexer_sm100_kernel<16, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
   }
   return check_launch("indexer_sm100_kernel");
 }
@@ -341,10 +370,19 @@ cslc_status launch_indexer_sm100(const uint16_t* q_idx, const uint16_t* w, const
                                  int L, int Nc, int HI, int m, int q_pos0, int row_begin, int row_end,
                                  void* scores, bool bf16_out, int rows_in_buf, cudaStream_t stream) {
   if (bf16_out)
-    return launch_indexer_sm100_t(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end,
-                                  static_cast<uint16_t*>(scores), rows_in_buf, stream);
-  return launch_indexer_sm100_t(q_idx, w, k_idx, B, L, Nc, HI, m, q_pos0, row_begin, row_end,
-                                static_cast<float*>(scores), rows_in_buf, stream);
+    return launch_indexer_sm100_t<uint16_t, false>(q_idx, w, k_idx, nullptr, nullptr, B, L, Nc, HI, m, q_pos0,
+                                                   row_begin, row_end, static_cast<uint16_t*>(scores), rows_in_buf,
+                                                   stream);
+  return launch_indexer_sm100_t<float, false>(q_idx, w, k_idx, nullptr, nullptr, B, L, Nc, HI, m, q_pos0, row_begin,
+                                              row_end, static_cast<float*>(scores), rows_in_buf, stream);
+}
+
+// e4m3 operands with per-row scales; fp32 scores [rows][Nc]
+cslc_status launch_indexer_sm100_fp8(const uint8_t* q8, const float* q_scale, const uint16_t* w, const uint8_t* k8,
+                                     const float* k_scale, int B, int L, int Nc, int HI, int m, int q_pos0,
+                                     int row_begin, int row_end, float* scores, int rows_in_buf, cudaStream_t stream) {
+  return launch_indexer_sm100_t<float, true>(q8, w, k8, q_scale, k_scale, B, L, Nc, HI, m, q_pos0, row_begin,
+                                             row_end, scores, rows_in_buf, stream);
 }
 
 int indexer_sm100_read_error() {

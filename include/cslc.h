@@ -202,6 +202,34 @@ cslc_status csa_indexer_topk_bf16(const cslc_bf16* q_idx, const cslc_bf16* w,
 cslc_status csa_topk_bf16(const cslc_bf16* scores, int B, int L, int Nc, int m, int q_pos0,
                           int topk, int32_t* idx, cslc_stream_t stream);
 
+/* FP8 indexer operands (first page §1.4: a low-precision lightning indexer).
+ *
+ * cslc_quantize_rows_e4m3: rows x [rows, d] bf16 -> codes [rows, d] uint8
+ * (e4m3) and scales [rows] fp32, per row s = amax(|x|) / 448 (1 for a zero
+ * row) and codes = RNE-saturate(x / s), scale and quotient in fp32 (the rule
+ * of cslc_quantize_kv_mixed). Requires d == 64 (the indexer's rows).
+ *
+ * csa_indexer_topk_fp8: csa_indexer_topk on e4m3 operands,
+ *   S[b,t,i] = sum_h w[b,t,h] * max(0, qd[b,t,h,:] . kd[b,i,:]),
+ *   qd = e4m3(q8) * q_scale[b,t,h],  kd = e4m3(k8) * k_scale[b,i],
+ * with the code products accumulated in fp32 on the tensor cores, the scales
+ * applied afterwards (they are positive: S = k_scale * sum_h w q_scale
+ * max(0, q8 . k8)), and the scores stored fp32; idx is their exact top-k
+ * under the rule of csa_indexer_topk.
+ *   q8 [B, L, H_I, 64] uint8, q_scale [B, L, H_I] fp32, w [B, L, H_I] bf16,
+ *   k8 [B, Nc, 64] uint8, k_scale [B, Nc] fp32 (scales > 0, as produced by
+ *   cslc_quantize_rows_e4m3), q8 and k8 16-byte aligned;
+ *   scores, idx, ws and ordering as csa_indexer_topk, workspace
+ *   csa_indexer_topk_workspace_bytes().
+ * Requires H_I in {1, 2, 4, 8, 16} and the other limits of csa_indexer_topk.
+ */
+cslc_status cslc_quantize_rows_e4m3(const cslc_bf16* x, int64_t rows, int d, uint8_t* codes, float* scales,
+                                    cslc_stream_t stream);
+cslc_status csa_indexer_topk_fp8(const uint8_t* q8, const float* q_scale, const cslc_bf16* w,
+                                 const uint8_t* k8, const float* k_scale, int B, int L, int Nc, int HI,
+                                 int dI, int m, int q_pos0, int topk, float* scores, int32_t* idx,
+                                 void* ws, size_t ws_bytes, cslc_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* CSA core attention ("读完这篇…" §三 注意力计算: ordinary attention over the
  * selected entries, KV shared by the heads)
