@@ -117,13 +117,23 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_scores_kernel(
   // 16tq+4s (+0,+1) and 16tq+4s+2 (+2,+3) -- the same pairs its B registers hold.
   const int c1 = min(n, c0 + DEC_CHUNK);
   const uint16_t* kbase = k_idx + (size_t)b * n_max * kDI;
-  for (int e0 = c0 + warp * 16; e0 < c1; e0 += 16 * (DEC_THREADS / 32)) {
+  // the key rows of a warp's group of 16 entries (clamped to the last entry);
+  // the next group's loads are issued before this group is used, so that two
+  // groups per warp are in flight
+  auto load_group = [&](int e0, uint4 (&v)[4]) {
+    const uint4* pa = reinterpret_cast<const uint4*>(kbase + (size_t)min(e0 + g, n - 1) * kDI + 16 * tq);
+    const uint4* pb = reinterpret_cast<const uint4*>(kbase + (size_t)min(e0 + g + 8, n - 1) * kDI + 16 * tq);
+    v[0] = __ldcs(pa); v[1] = __ldcs(pa + 1); v[2] = __ldcs(pb); v[3] = __ldcs(pb + 1);
+  };
+  constexpr int GROUP_STRIDE = 16 * (DEC_THREADS / 32);
+  uint4 nxt[4];
+  if (c0 + warp * 16 < c1) load_group(c0 + warp * 16, nxt);
+  for (int e0 = c0 + warp * 16; e0 < c1; e0 += GROUP_STRIDE) {
     const int ea = e0 + g, eb = ea + 8;
     uint32_t ra[8], rb[8];
     {
-      const uint4* pa = reinterpret_cast<const uint4*>(kbase + (size_t)min(ea, n - 1) * kDI + 16 * tq);
-      const uint4* pb = reinterpret_cast<const uint4*>(kbase + (size_t)min(eb, n - 1) * kDI + 16 * tq);
-      const uint4 a0 = __ldcs(pa), a1 = __ldcs(pa + 1), b0 = __ldcs(pb), b1 = __ldcs(pb + 1);
+      const uint4 a0 = nxt[0], a1 = nxt[1], b0 = nxt[2], b1 = nxt[3];
+      if (e0 + GROUP_STRIDE < c1) load_group(e0 + GROUP_STRIDE, nxt);
       ra[0] = a0.x; ra[1] = a0.y; ra[2] = a0.z; ra[3] = a0.w; ra[4] = a1.x; ra[5] = a1.y; ra[6] = a1.z; ra[7] = a1.w;
       rb[0] = b0.x; rb[1] = b0.y; rb[2] = b0.z; rb[3] = b0.w; rb[4] = b1.x; rb[5] = b1.y; rb[6] = b1.z; rb[7] = b1.w;
     }
