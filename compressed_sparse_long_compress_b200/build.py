@@ -67,7 +67,9 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = N
         for s, log in ex.map(compile_one, todo):
             if verbose_ptxas and log:
                 sys.stderr.write(f"== {os.path.basename(s)}\n{log}")
-    if todo or force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
+    # relink also when a source was added or removed (the directory changed)
+    newest = max([os.path.getmtime(o) for o in objs] + [os.path.getmtime(CSRC)])
+    if todo or force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
         cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-cudart", "static", *objs, "-o", LIB + ".tmp"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:

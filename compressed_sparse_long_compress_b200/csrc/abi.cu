@@ -38,10 +38,10 @@ cslc_status launch_indexer_scores(const uint16_t*, const uint16_t*, const uint16
                                   int, int, int, int, void*, bool, int, cudaStream_t);
 cslc_status launch_topk_rows(const void*, bool, int, int, int, int, int, int, int, int, int, int32_t*,
                              cudaStream_t);
-cslc_status launch_sparse_attn(const uint16_t*, const uint16_t*, const int32_t*, int, int, int, int, int,
-                               float, uint16_t*, float*, cudaStream_t);
-cslc_status launch_dense_attn(const uint16_t*, const uint16_t*, int, int, int, int, int, int, float,
-                              uint16_t*, float*, cudaStream_t);
+cslc_status launch_sparse_attn_sm100(const uint16_t*, const uint16_t*, const int32_t*, int, int, int, int, int,
+                                     float, uint16_t*, float*, cudaStream_t);
+cslc_status launch_dense_attn_sm100(const uint16_t*, const uint16_t*, int, int, int, int, int, int, float,
+                                    uint16_t*, float*, cudaStream_t);
 size_t decode_workspace_bytes(const cslc_decode_layer*, int, int, int);
 int sparse_attn_sm100_read_error();
 int dense_attn_sm100_read_error();
@@ -387,7 +387,7 @@ cslc_status csa_sparse_attn(const cslc_bf16* q, const cslc_bf16* kv, const int32
   REQUIRE_PTR(q); REQUIRE_PTR(idx); REQUIRE_PTR(out);
   if (Nc > 0) REQUIRE_PTR(kv);
   if (lse) REQUIRE_PTR(lse);
-  return launch_sparse_attn(q, kv, idx, B, L, H, Nc, topk, scale, out, lse, stream);
+  return launch_sparse_attn_sm100(q, kv, idx, B, L, H, Nc, topk, scale, out, lse, stream);
 }
 
 cslc_status hca_dense_attn(const cslc_bf16* q, const cslc_bf16* kv, int B, int L, int H, int D, int Nc,
@@ -402,7 +402,7 @@ cslc_status hca_dense_attn(const cslc_bf16* q, const cslc_bf16* kv, int B, int L
   REQUIRE_PTR(q); REQUIRE_PTR(out);
   if (Nc > 0) REQUIRE_PTR(kv);
   if (lse) REQUIRE_PTR(lse);
-  return launch_dense_attn(q, kv, B, L, H, Nc, m_prime, q_pos0, scale, out, lse, stream);
+  return launch_dense_attn_sm100(q, kv, B, L, H, Nc, m_prime, q_pos0, scale, out, lse, stream);
 }
 
 cslc_status cslc_quantize_kv_mixed(const cslc_bf16* kv, int B, int N, uint8_t* nope, cslc_bf16* rope,

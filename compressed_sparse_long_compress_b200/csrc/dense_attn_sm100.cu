@@ -5,7 +5,7 @@
 // window has ended, n_vis(t) = min(Nc, floor((t+1)/m')). K = V = the entry.
 //
 // Rows of the MMA are (token, head) pairs: a Q tile is 128 consecutive rows of
-// q viewed as [B*L*H, 128] (128/H tokens), loaded with one 2-D TMA per 64-dim
+// q viewed as [B*L tokens][H heads][128] (128/H tokens), loaded with one 3-D TMA per 64-dim
 // half. KV tiles are 128 consecutive entries (2-D TMA); the same shared tile is
 // K (K-major) for S = Q K^T and V (MN-major) for O += P V.
 //
@@ -65,7 +65,8 @@ struct DaSmall {
 
 __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
     int B, int L, int H, int Nc, int m, int q_pos0, float scale_log2, uint16_t* __restrict__ out,
-    float* __restrict__ lse, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv) {
+    float* __restrict__ lse, int h_stride, int h_off, const __grid_constant__ CUtensorMap tm_q,
+    const __grid_constant__ CUtensorMap tm_kv) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;                                   // [2 kb][128][128 B]
@@ -120,9 +121,10 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
         if (tk >= 1 && !mbar_wait(&bars.q_empty, (uint32_t)((tk - 1) & 1), abortp, errp, ERR_Q_EMPTY)) break;
         q_last = tk;
         mbar_arrive_expect_tx(&bars.q_full, DA_TILE_BYTES);
-        const int qrow = (int)(((long long)b * L + t0) * H);
-        tma_load_2d(q_s, &tm_q, 0, qrow, &bars.q_full);
-        tma_load_2d(q_s + DA_TILE * 128, &tm_q, 64, qrow, &bars.q_full);
+        // heads h_off .. h_off+H-1 of tokens t0 .. t0+128/H-1 (rows token-major)
+        const int tok0 = (int)((long long)b * L + t0);
+        tma_load_3d(q_s, &tm_q, 0, h_off, tok0, &bars.q_full);
+        tma_load_3d(q_s + DA_TILE * 128, &tm_q, 64, h_off, tok0, &bars.q_full);
         for (int j = 0; j < nkv; ++j) {
           const int stage = kv_it % DA_STAGES;
           if (kv_it >= DA_STAGES &&
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
       if (!ok) break;
       tc_fence_after();
       const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
-      const long long orow = ((long long)b * L + t0) * H + row;
+      const long long orow = ((long long)b * L + t0 + row / H) * h_stride + h_off + row % H;
 #pragma unroll
       for (int c0 = 0; c0 < 128; c0 += 32) {
         uint32_t r[32];
@@ -360,7 +362,10 @@ __global__ void __launch_bounds__(DA_THREADS, 1) dense_attn_sm100_kernel(
   }
 }
 
-bool dense_attn_sm100_supported(int H) { return H == 16 || H == 32 || H == 64 || H == 128; }
+// Any multiple of 16 up to 128 heads: groups of 128, 64, 32 and 16 heads (a
+// group's 128-row tiles hold whole tokens), one launch each on the group's
+// heads of q / out / lse.
+bool dense_attn_sm100_supported(int H) { return H >= 16 && H <= 128 && H % 16 == 0; }
 
 cslc_status launch_dense_attn_sm100(const uint16_t* q, const uint16_t* kv, int B, int L, int H, int Nc, int m,
                                     int q_pos0, float scale, uint16_t* out, float* lse, cudaStream_t stream) {
@@ -374,17 +379,26 @@ cslc_status launch_dense_attn_sm100(const uint16_t* q, const uint16_t* kv, int B
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     configured_for = dev;
   }
-  const int tpt = DA_ROWS / H;
-  const long long n_qt = (long long)B * ((L + tpt - 1) / tpt);
-  const int grid = (int)(n_qt < n_sm ? n_qt : n_sm);
-  CUtensorMap tm_q, tm_kv;
   const void* kv_base = Nc > 0 ? (const void*)kv : (const void*)q;
-  if (!sm100::make_tmap_bf16_2d(&tm_q, q, (uint64_t)B * L * H, kD, kD * 2, DA_ROWS, 64) ||
-      !sm100::make_tmap_bf16_2d(&tm_kv, kv_base, (uint64_t)B * (Nc > 0 ? Nc : 1), kD, kD * 2, DA_TILE, 64))
+  CUtensorMap tm_kv;
+  if (!sm100::make_tmap_bf16_2d(&tm_kv, kv_base, (uint64_t)B * (Nc > 0 ? Nc : 1), kD, kD * 2, DA_TILE, 64))
     return set_error(CSLC_ERR_CUDA, "hca_dense_attn: tensor map encoding failed");
-  dense_attn_sm100_kernel<<<grid, DA_THREADS, smem, stream>>>(B, L, H, Nc, m, q_pos0, scale * kLog2e, out, lse,
-                                                              tm_q, tm_kv);
-  return check_launch("dense_attn_sm100_kernel");
+  for (int h0 = 0; h0 < H;) {
+    const int rem = H - h0;
+    const int hg = rem >= 128 ? 128 : rem >= 64 ? 64 : rem >= 32 ? 32 : 16;
+    const int tpt = DA_ROWS / hg;
+    const long long n_qt = (long long)B * ((L + tpt - 1) / tpt);
+    const int grid = (int)(n_qt < n_sm ? n_qt : n_sm);
+    CUtensorMap tm_q;   // q as [B*L tokens][H heads][128]; a box is 64 dims x hg heads x 128/hg tokens
+    if (!sm100::make_tmap_bf16_3d(&tm_q, q, (uint64_t)H, (uint64_t)B * L, (uint32_t)hg, (uint32_t)tpt))
+      return set_error(CSLC_ERR_CUDA, "hca_dense_attn: tensor map encoding failed");
+    dense_attn_sm100_kernel<<<grid, DA_THREADS, smem, stream>>>(B, L, hg, Nc, m, q_pos0, scale * kLog2e, out, lse, H,
+                                                                h0, tm_q, tm_kv);
+    const cslc_status st = check_launch("dense_attn_sm100_kernel");
+    if (st != CSLC_OK) return st;
+    h0 += hg;
+  }
+  return CSLC_OK;
 }
 
 int dense_attn_sm100_read_error() {

@@ -256,6 +256,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 // Row gather: four rows y0..y3 (box one row high, columns x .. x+box-1)
 // land as four consecutive box rows in shared memory. Rows outside the
 // tensor read the zero fill.
@@ -301,6 +308,9 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 
 // box_rows x box_cols elements and 128-byte swizzle; false on failure.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_pitch_bytes,
                        uint32_t box_rows, uint32_t box_cols);
+// [n2][n1][128] bf16 (rows of 256 B, n1 rows per outer index), 128-byte swizzle,
+// boxes of 64 x box1 x box2
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n1, uint64_t n2, uint32_t box1, uint32_t box2);
 // rows of 64 bytes (e4m3 codes), 64-byte swizzle, boxes of box_rows x 64
 bool make_tmap_u8_rows64(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows);
 

@@ -133,7 +133,7 @@ template <int H>
 __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ kv, const int32_t* __restrict__ idx,
     int B, int L, int Nc, int topk, float scale_log2, uint16_t* __restrict__ out, float* __restrict__ lse,
-    const __grid_constant__ CUtensorMap tm_q) {
+    int h_stride, int h_off, const __grid_constant__ CUtensorMap tm_q) {
   constexpr int HT = H / 2;           // heads per softmax thread
   static_assert(HT % 8 == 0 && HT <= 32, "H must be 16, 32 or 64");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -220,8 +220,9 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
         sm->ref_slot[qb] = min(min(sm->first_w[qb][0], sm->first_w[qb][1]), sm->first_w[qb][2]);
         uint8_t* qd = q_s + qb * SA_Q_BYTES;
         mbar_arrive_expect_tx(&bars.tok_full[qb], (uint32_t)(H * 256));
-        tma_load_2d(qd, &tm_q, 0, (int)(g * H), &bars.tok_full[qb]);
-        tma_load_2d(qd + SA_NP * 128, &tm_q, 64, (int)(g * H), &bars.tok_full[qb]);
+        const int qrow = (int)(g * h_stride + h_off);   // this token's first head of the group
+        tma_load_2d(qd, &tm_q, 0, qrow, &bars.tok_full[qb]);
+        tma_load_2d(qd + SA_NP * 128, &tm_q, 64, qrow, &bars.tok_full[qb]);
         if (qb == 0) q_issued0 = tk; else q_issued1 = tk;
       }
       const uint16_t* kvb = kv + (g / L) * (long long)Nc * kD;
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
       if (tid < H) {
         const float l = sm->red[0][tid] + sm->red[1][tid] + sm->red[2][tid] + sm->red[3][tid];
         sm->inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
-        if (lse != nullptr) lse[g * H + tid] = l > 0.f ? (sm->mref[tid] + log2f(l)) * kLn2 : -INFINITY;
+        if (lse != nullptr) lse[g * h_stride + h_off + tid] = l > 0.f ? (sm->mref[tid] + log2f(l)) * kLn2 : -INFINITY;
       }
       {
         bool w = true;
@@ -477,7 +478,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) sparse_attn_sm100_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.o_free[ob]);
       named_bar(2, SA_NSOFT);
-      uint4* dst = reinterpret_cast<uint4*>(out + g * (long long)H * kD);
+      uint4* dst = reinterpret_cast<uint4*>(out + (g * (long long)h_stride + h_off) * kD);
       const uint4* src = reinterpret_cast<const uint4*>(stage_out);
       for (int x = tid; x < H * 16; x += SA_NSOFT) dst[x] = src[x];
       named_bar(2, SA_NSOFT);
@@ -568,7 +569,10 @@ constexpr size_t sa_smem_bytes() {
 }
 }  // namespace
 
-bool sparse_attn_sm100_supported(int H) { return H == 16 || H == 32 || H == 64; }
+// Any multiple of 16 up to 128 heads: groups of 64, 32 and 16 heads, one
+// launch each on a view of q / out / lse that starts at the group's first
+// head (the gathered entries are read again by every group, from L2).
+bool sparse_attn_sm100_supported(int H) { return H >= 16 && H <= 128 && H % 16 == 0; }
 
 cslc_status launch_sparse_attn_sm100(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int L,
                                      int H, int Nc, int topk, float scale, uint16_t* out, float* lse,
@@ -588,15 +592,21 @@ cslc_status launch_sparse_attn_sm100(const uint16_t* q, const uint16_t* kv, cons
   const long long n_tok = (long long)B * L;
   const int grid = (int)(n_tok < n_sm ? n_tok : n_sm);
   const float sl2 = scale * kLog2e;
-  CUtensorMap tm_q;   // q viewed as [B*L*H rows, 128] with a box of H rows x 64 dims
-  if (!sm100::make_tmap_bf16_2d(&tm_q, q, (uint64_t)n_tok * H, kD, kD * 2, (uint32_t)H, 64))
-    return set_error(CSLC_ERR_CUDA, "csa_sparse_attn: tensor map encoding failed");
-  switch (H) {
-    case 16: sparse_attn_sm100_kernel<16><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, tm_q); break;
-    case 32: sparse_attn_sm100_kernel<32><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, tm_q); break;
-    default: sparse_attn_sm100_kernel<64><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, tm_q); break;
+  for (int h0 = 0; h0 < H;) {
+    const int hg = H - h0 >= 64 ? 64 : (H - h0 >= 32 ? 32 : 16);
+    CUtensorMap tm_q;   // q viewed as [B*L*H rows, 128] with a box of hg rows x 64 dims
+    if (!sm100::make_tmap_bf16_2d(&tm_q, q, (uint64_t)n_tok * H, kD, kD * 2, (uint32_t)hg, 64))
+      return set_error(CSLC_ERR_CUDA, "csa_sparse_attn: tensor map encoding failed");
+    switch (hg) {
+      case 16: sparse_attn_sm100_kernel<16><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, H, h0, tm_q); break;
+      case 32: sparse_attn_sm100_kernel<32><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, H, h0, tm_q); break;
+      default: sparse_attn_sm100_kernel<64><<<grid, SA_THREADS, smem, stream>>>(q, kv, idx, B, L, Nc, topk, sl2, out, lse, H, h0, tm_q); break;
+    }
+    const cslc_status st = check_launch("sparse_attn_sm100_kernel");
+    if (st != CSLC_OK) return st;
+    h0 += hg;
   }
-  return check_launch("sparse_attn_sm100_kernel");
+  return CSLC_OK;
 }
 
 int sparse_attn_sm100_read_error() {

@@ -229,6 +229,8 @@ def _random_idx(rng, L, n_c, topk, holes=False):
 @pytest.mark.parametrize("H,L,n_c,topk,holes,q_scale", [
     (16, 512, 1024, 128, False, 1.0), (64, 128, 16384, 1024, False, 1.0), (128, 64, 3000, 200, True, 1.0),
     (64, 96, 2000, 1000, True, 8.0), (16, 40, 10, 2048, False, 1.0),
+    # head counts run as groups of 64 / 32 / 16 heads
+    (48, 200, 3000, 256, True, 1.0), (112, 64, 2000, 512, False, 8.0), (80, 33, 500, 300, True, 1.0),
 ])
 def test_sparse_attention_isolated(C, H, L, n_c, topk, holes, q_scale):
     rng = np.random.default_rng(H + L)
@@ -248,6 +250,8 @@ def test_sparse_attention_isolated(C, H, L, n_c, topk, holes, q_scale):
 @pytest.mark.parametrize("H,L,m,n_c,q_pos0,q_scale", [
     (16, 4096, 128, 32, 0, 1.0), (64, 1001, 4, 250, 0, 1.0), (128, 300, 4, 2000, 5000, 1.0),
     (64, 513, 128, 40, 4000, 8.0), (16, 50, 1, 50, 0, 1.0),
+    # head counts run as groups of 128 / 64 / 32 / 16 heads
+    (48, 700, 4, 200, 0, 1.0), (80, 301, 128, 40, 4000, 8.0), (96, 513, 4, 128, 0, 1.0), (112, 130, 2, 90, 7, 1.0),
 ])
 def test_dense_attention_isolated(C, H, L, m, n_c, q_pos0, q_scale):
     q = W.randn_bf16((1, L, H, 128), 51)
@@ -291,7 +295,7 @@ def test_attention_with_scores_growing_along_the_entries(C, H):
     assert_close_scaled(f64(lse_s), l_ref, what="sparse attn lse (growing)")
 
 
-@pytest.mark.parametrize("H", [64, 128])
+@pytest.mark.parametrize("H", [64, 128, 48])
 def test_sparse_attention_two_sequences(C, H):
     # B = 2: each sequence's index rows select from its own entries
     L, n_c, topk = 150, 1500, 600
@@ -306,7 +310,7 @@ def test_sparse_attention_two_sequences(C, H):
     assert_close(f64(lse), l_ref, what="sparse attn lse (B=2)")
 
 
-@pytest.mark.parametrize("H,q_pos0", [(64, 0), (16, 700)])
+@pytest.mark.parametrize("H,q_pos0", [(64, 0), (16, 700), (96, 5), (48, 0)])
 def test_dense_attention_two_sequences(C, H, q_pos0):
     # B = 2 with a ragged L: the last query tile of a sequence runs past its end
     L, m = 333, 4
