@@ -242,7 +242,6 @@ static cslc_status indexer_topk_impl(const char* fn, const IndexerOperands& op, 
   REQUIRE(B >= 0 && L >= 0 && Nc >= 0 && q_pos0 >= 0 && m >= 1, CSLC_ERR_SHAPE, "%s: negative size / m < 1", fn);
   REQUIRE(dI == kDI, CSLC_ERR_UNSUPPORTED, "%s: d_I must be 64 (got %d)", fn, dI);
   REQUIRE(HI >= 1 && HI <= 16, CSLC_ERR_UNSUPPORTED, "%s: H_I must be in [1, 16]", fn);
-  REQUIRE(!op.fp8 || is_pow2(HI), CSLC_ERR_UNSUPPORTED, "%s: H_I must be 1, 2, 4, 8 or 16 (got %d)", fn, HI);
   REQUIRE(topk >= 1 && topk <= kMaxTopk, CSLC_ERR_UNSUPPORTED, "%s: topk must be in [1, 2048]", fn);
   REQUIRE(Nc <= kMaxPrefillTopkNc, CSLC_ERR_UNSUPPORTED, "%s: Nc must be <= %d", fn, kMaxPrefillTopkNc);
   if ((long long)B * L == 0) return CSLC_OK;

@@ -6,12 +6,14 @@
 //
 // One MMA tile is D = K_I E^T with
 //   A = 128 consecutive entries of k_I           (128 x d_I, K-major, TMA)
-//   B = 256 consecutive (token, head) rows of q_I viewed as [B*L*H_I, d_I]
-//       (256 / H_I tokens, K-major, TMA)
+//   B = 256 (token, head) rows of q_I: 256 / HP tokens x HP heads, where HP is
+//       H_I rounded up to a power of two (a 3-D TMA over tokens x heads x
+//       dims fills the heads past H_I with zeros; their weights are zero)
 // so D (fp32, in TMEM) holds entry i in lane i and pair (t, h) in column
-// t*H_I + h: the weighted ReLU head sum of a score is a sum over H_I adjacent
+// t*HP + h: the weighted ReLU head sum of a score is a sum over HP adjacent
 // columns inside one thread, and a warp's 32 lanes store 32 consecutive
-// entries of one score row (128-byte stores).
+// entries of one score row (128-byte stores). Boxes reaching past the end of
+// q_I or k_I read zeros, so any size runs on this kernel.
 //
 // CTA roles (persistent, one CTA per SM; work items = a query-row tile and a
 // chunk of 16 key tiles, heavy rows first, dealt to the CTAs in a snake so that
@@ -85,11 +87,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void store_score(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_score(uint16_t* p, float v) { *p = __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
-template <int HI, typename OutT, bool FP8>
+template <int HI, typename OutT, bool FP8>   // HI: heads per token in a tile (H_I rounded up to a power of two)
 __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
     const uint16_t* __restrict__ w, const float* __restrict__ q_scale, const float* __restrict__ k_scale, int B,
-    int L, int Nc, int m, int q_pos0, int row_begin, int row_end, OutT* __restrict__ scores, int rows_in_buf,
-    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
+    int L, int Nc, int HI_act, int m, int q_pos0, int row_begin, int row_end, OutT* __restrict__ scores,
+    int rows_in_buf, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
   constexpr int RT = IX_NP / HI;                 // query rows per tile
   // bytes of a loaded tile (the shared-memory slots are sized for bf16)
   constexpr uint32_t Q_TX = FP8 ? IX_NP * 64 : IX_Q_BYTES, K_TX = FP8 ? IX_ET * 64 : IX_K_BYTES;
@@ -109,7 +111,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
   const int et_max = (n_visible((long long)q_pos0 + row_end - 1, m, Nc) + IX_ET - 1) / IX_ET;
   const int n_ch = max(1, (et_max + IX_CHUNK - 1) / IX_CHUNK);
   const int n_items = B * rt_per_b * n_ch;
-  const long long n_pairs = (long long)B * L * HI;
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -162,12 +163,13 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       if (lane == 0 && rq >= 2)
         w_ok = mbar_wait(&bars.q_empty[qs], (uint32_t)(((rq >> 1) - 1) & 1), abortp, errp, ERR_Q_EMPTY);
       if (!__shfl_sync(0xffffffffu, (int)w_ok, 0)) break;
-      const long long p0 = ((long long)b * L + t0) * HI;
 #pragma unroll
       for (int x = 0; x < IX_NP / 32; ++x) {
-        const long long p = p0 + x * 32 + lane;
-        float wv = p < n_pairs ? bf16_to_f(w[p]) : 0.f;
-        if constexpr (FP8) wv *= p < n_pairs ? q_scale[p] : 0.f;
+        const int j = x * 32 + lane, t = t0 + j / HI, h = j % HI;   // pair j of the tile
+        const bool real = h < HI_act && t < L;                     // padding heads and rows past L weigh 0
+        const long long p = ((long long)b * L + t) * HI_act + h;
+        float wv = real ? bf16_to_f(w[p]) : 0.f;
+        if constexpr (FP8) wv *= real ? q_scale[p] : 0.f;
         w_s[qs * IX_NP + x * 32 + lane] = wv;
       }
       for (int r = lane; r < RT; r += 32)
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&bars.q_full[qs], Q_TX);
-        tma_load_2d(q_s + qs * IX_Q_BYTES, &tm_q, 0, (int)p0, &bars.q_full[qs]);
+        tma_load_3d(q_s + qs * IX_Q_BYTES, &tm_q, 0, 0, b * L + t0, &bars.q_full[qs]);
         for (int et = et0; et < et0 + n_et; ++et, ++kt) {
           const int ks = kt % IX_KSTAGES;
           if (kt >= IX_KSTAGES &&
@@ -321,8 +323,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_sm100_kernel(
   }
 }
 
-bool indexer_sm100_supported(int HI) { return HI == 1 || HI == 2 || HI == 4 || HI == 8 || HI == 16; }
-
 template <typename OutT, bool FP8>
 static cslc_status launch_indexer_sm100_t(const void* q_idx, const uint16_t* w, const void* k_idx,
                                           const float* q_scale, const float* k_scale, int B, int L, int Nc, int HI,
@@ -343,24 +343,25 @@ static cslc_status launch_indexer_sm100_t(const void* q_idx, const uint16_t* w, 
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     configured_for = dev;
   }
-  const int RT = IX_NP / HI;
+  const int HP = HI <= 1 ? 1 : HI <= 2 ? 2 : HI <= 4 ? 4 : HI <= 8 ? 8 : 16;
+  const int RT = IX_NP / HP;
   const int et_max = (n_visible((long long)q_pos0 + row_end - 1, m, Nc) + IX_ET - 1) / IX_ET;
   const int n_ch = et_max > IX_CHUNK ? (et_max + IX_CHUNK - 1) / IX_CHUNK : 1;
   const int n_items = B * ((row_end - row_begin + RT - 1) / RT) * n_ch;
   const int grid = n_items < n_sm ? n_items : n_sm;
   CUtensorMap tm_q, tm_k;
+  const int eb = FP8 ? 1 : 2;   // bytes per element; a row is 64 elements
   const bool maps_ok =
-      FP8 ? make_tmap_u8_rows64(&tm_q, q_idx, (uint64_t)B * L * HI, IX_NP) &&
-                make_tmap_u8_rows64(&tm_k, k_idx, (uint64_t)B * Nc, IX_ET)
-          : make_tmap_bf16_2d(&tm_q, q_idx, (uint64_t)B * L * HI, kDI, kDI * 2, IX_NP, 64) &&
-                make_tmap_bf16_2d(&tm_k, k_idx, (uint64_t)B * Nc, kDI, kDI * 2, IX_ET, 64);
+      make_tmap_rows3d(&tm_q, q_idx, eb, (uint64_t)HI, (uint64_t)B * L, (uint32_t)HP, (uint32_t)RT) &&
+      (FP8 ? make_tmap_u8_rows64(&tm_k, k_idx, (uint64_t)B * Nc, IX_ET)
+           : make_tmap_bf16_2d(&tm_k, k_idx, (uint64_t)B * Nc, kDI, kDI * 2, IX_ET, 64));
   if (!maps_ok) return set_error(CSLC_ERR_CUDA, "csa_indexer_topk: tensor map encoding failed");
-  switch (HI) {
-    case 1: indexer_sm100_kernel<1, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 2: indexer_sm100_kernel<2, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 4: indexer_sm100_kernel<4, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    case 8: indexer_sm100_kernel<8, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
-    default: indexer_sm100_kernel<16, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+  switch (HP) {
+    case 1: indexer_sm100_kernel<1, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 2: indexer_sm100_kernel<2, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 4: indexer_sm100_kernel<4, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    case 8: indexer_sm100_kernel<8, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
+    default: indexer_sm100_kernel<16, OutT, FP8><<<grid, IX_THREADS, smem, stream>>>(w, q_scale, k_scale, B, L, Nc, HI, m, q_pos0, row_begin, row_end, scores, rows_in_buf, tm_q, tm_k); break;
   }
   return check_launch("indexer_sm100_kernel");
 }

@@ -311,6 +311,10 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 // [n2][n1][128] bf16 (rows of 256 B, n1 rows per outer index), 128-byte swizzle,
 // boxes of 64 x box1 x box2
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n1, uint64_t n2, uint32_t box1, uint32_t box2);
+// [n2][n1][64] rows of 64 elements of eb bytes (bf16: 128-byte rows, 128-byte
+// swizzle; e4m3: 64-byte rows, 64-byte swizzle), boxes of 64 x box1 x box2
+bool make_tmap_rows3d(CUtensorMap* map, const void* base, int eb, uint64_t n1, uint64_t n2, uint32_t box1,
+                      uint32_t box2);
 // rows of 64 bytes (e4m3 codes), 64-byte swizzle, boxes of box_rows x 64
 bool make_tmap_u8_rows64(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows);
 

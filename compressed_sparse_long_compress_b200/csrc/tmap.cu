@@ -49,6 +49,22 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t n1, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_rows3d(CUtensorMap* map, const void* base, int eb, uint64_t n1, uint64_t n2, uint32_t box1,
+                      uint32_t box2) {
+  auto fn = encode_fn();
+  if (fn == nullptr || (eb != 1 && eb != 2)) return false;
+  const cuuint64_t row = 64ull * eb;
+  const cuuint64_t dims[3] = {64, n1, n2};
+  const cuuint64_t strides[2] = {row, row * n1};
+  const cuuint32_t box[3] = {64, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        eb == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_u8_rows64(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;

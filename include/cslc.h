@@ -221,7 +221,7 @@ cslc_status csa_topk_bf16(const cslc_bf16* scores, int B, int L, int Nc, int m, 
  *   cslc_quantize_rows_e4m3), q8 and k8 16-byte aligned;
  *   scores, idx, ws and ordering as csa_indexer_topk, workspace
  *   csa_indexer_topk_workspace_bytes().
- * Requires H_I in {1, 2, 4, 8, 16} and the other limits of csa_indexer_topk.
+ * Requires the limits of csa_indexer_topk.
  */
 cslc_status cslc_quantize_rows_e4m3(const cslc_bf16* x, int64_t rows, int d, uint8_t* codes, float* scales,
                                     cslc_stream_t stream);

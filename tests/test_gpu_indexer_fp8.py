@@ -49,6 +49,7 @@ def _fp8_inputs(C, B, L, Nc, HI, seed):
 @pytest.mark.parametrize("B,L,HI,m,topk,q_pos0,Nc", [
     (1, 4096, 8, 4, 1024, 0, 1024), (2, 1001, 4, 4, 128, 0, 250), (1, 777, 16, 2, 64, 300, 700),
     (1, 1500, 1, 4, 32, 0, 375), (1, 640, 2, 4, 100, 0, 160), (1, 10, 2, 4, 8, 0, 40),
+    (2, 500, 6, 4, 64, 0, 125), (1, 300, 11, 2, 30, 5, 160),
 ])
 def test_fp8_indexer_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
     q, k, w, q8, qs, k8, ks = _fp8_inputs(C, B, L, Nc, HI, 1510 + L)

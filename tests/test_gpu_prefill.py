@@ -104,8 +104,11 @@ def _indexer_case(C, B, L, HI, m, topk, q_pos0, wid, Nc=None):
     (1, 777, 16, 4, 100, 37, None),         # 16 indexer heads, query offset
     (1, 512, 1, 2, 300, 0, None),           # k above most rows' visible counts
     (1, 300, 8, 4, 2048, 4000, 1100),       # later queries of a longer sequence
-    (1, 700, 6, 4, 64, 0, None),            # H_I not a power of two (mma.sync kernel)
-    (1, 40, 4, 4, 16, 0, None),             # fewer than 256 query pairs (mma.sync kernel)
+    (1, 700, 6, 4, 64, 0, None),            # H_I not a power of two (heads padded to 8 with zeros)
+    (2, 333, 3, 4, 50, 0, None),            # H_I = 3 (padded to 4), two sequences
+    (1, 257, 12, 2, 40, 9, None),           # H_I = 12 (padded to 16), query offset
+    (1, 40, 4, 4, 16, 0, None),             # fewer than 256 query pairs (boxes past the end read zeros)
+    (1, 9, 5, 4, 4, 0, None),               # 2 entries, 5 heads: every box mostly past the end
 ])
 def test_indexer_topk_matches_oracle(C, B, L, HI, m, topk, q_pos0, Nc):
     x, idx, idx_blocked, sc = _indexer_case(C, B, L, HI, m, topk, q_pos0, 31, Nc)
