@@ -675,11 +675,11 @@ def profile_case(name):
 # kernel source is the one that was measured.
 MEASURED_TRAFFIC = {
     "sparse": {"src": "sparse_attn_sm100.cu",
-               "sha256": "aef8a553ca588a590c3111df77e6cb1aedbe1e808e09b36955548148c2ee4bc2",
-               "bytes_per_token": (172.444416e6 + 101.987328e6) / 8192},
+               "sha256": "cda61cee7a0fdc35704200d66d5b4d744ea8af7d444108eee9d43312f00d39be",
+               "bytes_per_token": (172.049920e6 + 100.580352e6) / 8192},
     "dense": {"src": "dense_attn_sm100.cu",
-              "sha256": "288507378b3c15bc7d245eaa6a83a4535775efaf20ba08db79a0d8c7654f0086",
-              "bytes_per_token": (271.271424e6 + 221.559552e6) / 16384},
+              "sha256": "c973b4b6687b01d616c69815ea7577dcb6608b99ea5a390f0bafd7de8f99b29a",
+              "bytes_per_token": (271.014400e6 + 220.154624e6) / 16384},
 }
 
 
