@@ -100,3 +100,29 @@ def test_validation_decode_append():
     st, _ = _err(cslc.LIB.cslc_decode_append(P, P, P, P, P, P, P, 2, 4, 1, P, P, P, P, P, P, P, P, 8, P, P))
     assert st == 1   # c is NULL
     assert cslc.LIB.cslc_decode_append(P, P, P, P, P, P, P, 0, 4, 1, P, P, P, P, P, P, P, P, 8, P, P) == 0
+
+
+def test_fp8_entry_points_validation():
+    p = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1004)
+    # the row quantiser takes rows of 64 values only
+    st, msg = _err(cslc.LIB.cslc_quantize_rows_e4m3(p, 10, 128, p, p, None))
+    assert st == 4 and "d must be 64" in msg
+    st, _ = _err(cslc.LIB.cslc_quantize_rows_e4m3(p, -1, 64, p, p, None))
+    assert st == 2
+    assert cslc.LIB.cslc_quantize_rows_e4m3(None, 0, 64, None, None, None) == 0   # nothing to do
+    st, msg = _err(cslc.LIB.cslc_quantize_rows_e4m3(p, 10, 64, p, odd, None))
+    assert st == 3 and "scales" in msg
+    # FP8 indexer: scales are required, H_I in [1, 16], d_I = 64, workspace as the fp32 path
+    args = lambda qs, ks, HI, dI, ws, nbytes: (p, qs, p, p, ks, 1, 4096, 1024, HI, dI, 4, 0, 128, None, p, ws,
+                                                 nbytes, None)
+    st, msg = _err(cslc.LIB.csa_indexer_topk_fp8(*args(None, p, 8, 64, None, 0)))
+    assert st == 1 and "q_scale" in msg
+    st, msg = _err(cslc.LIB.csa_indexer_topk_fp8(*args(p, None, 8, 64, None, 0)))
+    assert st == 1 and "k_scale" in msg
+    st, _ = _err(cslc.LIB.csa_indexer_topk_fp8(*args(p, p, 17, 64, None, 0)))
+    assert st == 4
+    st, _ = _err(cslc.LIB.csa_indexer_topk_fp8(*args(p, p, 8, 32, None, 0)))
+    assert st == 4
+    st, msg = _err(cslc.LIB.csa_indexer_topk_fp8(*args(p, p, 6, 64, None, 0)))
+    assert st == 5 and "workspace" in msg   # H_I = 6 is accepted; only the workspace is missing
