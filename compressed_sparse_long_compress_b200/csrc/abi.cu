@@ -74,11 +74,12 @@ static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
   } while (0)
 
 // When the caller does not keep the scores they are produced in blocks of
-// this many rows, two blocks in flight: the top-k of one block runs on an
-// auxiliary stream beside the indexer of the next, so neither launch's tail
-// leaves SMs idle.
+// this many rows (up to 4 GiB of scores), two blocks in flight when there are
+// more: the top-k of one block runs on an auxiliary stream beside the indexer
+// of the next. Large blocks measured faster than small ones (fewer launch
+// tails), and one block, where it fits, faster than two side by side.
 static int score_block_rows(int Nc, int score_bytes = 4) {
-  const long long budget = 512ll << 20;   // bytes of scores per block
+  const long long budget = 4096ll << 20;   // bytes of scores per block
   long long rows = budget / ((long long)Nc * score_bytes);
   rows = rows < 64 ? 64 : rows;
   rows = (rows / 64) * 64;

@@ -138,7 +138,7 @@ def test_indexer_topk_blocks_in_flight(C):
     streams (three blocks here, so a buffer is reused): the selection equals
     the one made from the full score tensor, which the oracle checks on
     sampled rows."""
-    B, L, HI, m, topk, Nc = 1, 6000, 4, 4, 512, 45056
+    B, L, HI, m, topk, Nc = 1, 9000, 4, 4, 512, 262144   # 1 MB of scores per row
     q_pos0 = m * Nc - L
     block_bytes = C.indexer_topk_workspace_bytes(B, L, Nc, HI, topk) // 2   # two buffers
     rows_per_block = block_bytes // (B * Nc * 4)
