@@ -890,7 +890,6 @@ __global__ void __launch_bounds__(TAIL_THREADS) decode_tail_kernel(
     const uint32_t T = (uint32_t)s_thr[0];
     uint2* my_cand = cand + (size_t)b * n_max + e_lo;
     const float* srow = scores + (size_t)b * n_max;
-    const unsigned lt = (1u << lane) - 1u;
     // rounds of 32 scores per thread: flag masks (above the bin / in it),
     // one block scan of the counts, then each thread writes its scores' entry
     // numbers (above: this CTA's list; in the bin: its candidate slice)
