@@ -304,7 +304,7 @@ class FrontEnd:
         ach = self.flops / (kernel_ms * 1e-3) / 1e12
         return {"kernel": "compress_front_end (front_end_sm100_kernel<true>)", "bound": "tensor",
                 "achieved": round(ach, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": None,
+                "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": measured_traffic("front_end", self.units),
                 "algorithmic_flops_per_launch": self.flops, "peak_source": peaks["source"] + " (burst)"}
 
     def config(self):
@@ -352,7 +352,8 @@ class Decode:
     def roofline(self, kernel_ms, peaks):
         ach = self.bytes / (kernel_ms * 1e-3) / 1e9
         return {"kernel": "whole decode step (cslc_decode_step)", "bound": "hbm", "achieved": round(ach, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                "traffic": measured_traffic(self.name, 1),
                 "algorithmic_bytes_per_launch": self.bytes, "peak_source": peaks["source"]}
 
     def config(self):
@@ -680,6 +681,17 @@ MEASURED_TRAFFIC = {
     "dense": {"src": "dense_attn_sm100.cu",
               "sha256": "c973b4b6687b01d616c69815ea7577dcb6608b99ea5a390f0bafd7de8f99b29a",
               "bytes_per_token": (271.014400e6 + 220.154624e6) / 16384},
+    "front_end": {"src": "front_end_sm100.cu",
+                  "sha256": "5690b1b7653aa1670ccd6b0fa5174caa3af789ce22d347caf149faa33f399ac7",
+                  "bytes_per_token": (249.420800e6 + 3.766784e6) / 16384},
+    # decode: the DRAM bytes of one whole step (all its launches, serialised
+    # under ncu), so the unit is the step
+    "csa_decode": {"src": "decode.cu",
+                   "sha256": "79b227ff000d5a97fe43664dbc79b989fe701a21b6cf71614ea721f8ac94d586",
+                   "bytes_per_token": 305214464.0},
+    "hybrid_decode": {"src": "decode.cu",
+                      "sha256": "79b227ff000d5a97fe43664dbc79b989fe701a21b6cf71614ea721f8ac94d586",
+                      "bytes_per_token": 615825664.0},
 }
 
 
